@@ -1,0 +1,477 @@
+"""Benchmark of the HySparse MQA forward path on B200.
+
+One step = one pass of the whole forward path over one batch of synthetic
+input: hs_block_score -> hs_select_topk -> hs_sparse_mqa_fwd, plus
+hs_swa_mqa_fwd over the same q, k, v.  Default workload: one document of
+4096 tokens, 64 query heads over one KV head, Dk 576 (512 latent + 64 RoPE),
+Dv 512, bf16, block 64, top-16, window 512.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps; then K
+steps, each bracketed by CUDA events on the launching stream with an L2
+flush (a 512 MiB write) between steps outside the events; barrier +
+synchronize around the timed loop; max over ranks.  Under torchrun every
+rank runs its own replica of the workload (weak scaling, no data-path
+collective: documents are independent).
+
+``--impl reference`` times the float64 CPU oracle (the only reference this
+path has) on a bounded sample of query rows of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_mqa_b200 import hs, synth, workloads  # noqa: E402
+
+METRIC = "HySparse fwd tokens/s at 64 heads, Dk576/Dv512; % of bf16 tensor peak"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=workloads.MAIN.name)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=48,
+                    help="query rows of the oracle sample (cpu_baseline / reference arm)")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (valid (query, key) pairs only)
+# ---------------------------------------------------------------------------
+
+def causal_pairs(docs):
+    return sum(n * (n + 1) // 2 for n in docs)
+
+
+def window_pairs(docs, W):
+    tot = 0
+    for n in docs:
+        m = min(n, W)
+        tot += m * (m + 1) // 2 + (n - m) * W
+    return tot
+
+
+def sparse_pairs(idx, cu, B):
+    """sum_t |S_t| from the selected blocks (keys of each block up to t)."""
+    idx = idx.cpu().numpy().astype(np.int64)
+    tot = 0
+    for d in range(len(cu) - 1):
+        bos, eos = cu[d], cu[d + 1]
+        if eos <= bos:
+            continue
+        t = np.arange(bos, eos)[:, None]
+        b = idx[bos:eos]
+        lo = bos + b * B
+        cnt = np.minimum(lo + B, t + 1) - lo
+        tot += int(np.where(b >= 0, np.clip(cnt, 0, B), 0).sum())
+    return tot
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on a bounded sample (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(wl, rows_n, seed=0):
+    """Inputs and a row sample for the oracle (host tensors, same recipe)."""
+    import oracle.hysparse as O  # test infrastructure: the CPU baseline only
+    inp = synth.make_inputs(wl.total_tokens, wl.num_heads, wl.dk, wl.dv, dtype=wl.dtype,
+                            seed=seed, device="cpu", doc_lengths=wl.docs())
+    f = lambda t: t.double().numpy()
+    host = (f(inp.q), f(inp.k), f(inp.v), f(inp.sink), inp.cu_seqlens.tolist())
+    per_doc = max(2, rows_n // len(wl.docs()))
+    rows = synth.sample_rows(inp.cu_seqlens, per_doc, seed)
+    return O, host, rows
+
+
+def oracle_step(O, host, rows, wl):
+    q, k, v, s, cu = host
+    bs = O.block_score(q, k, cu, wl.block_size, rows=rows)
+    idx = O.select_topk(bs["block_score"], cu, wl.block_size, wl.topk, rows=rows,
+                        total_tokens=wl.total_tokens)
+    O.sparse_mqa_fwd(q, k, v, idx, cu, wl.block_size, sink=s, rows=rows)
+    O.swa_mqa_fwd(q, k, v, cu, wl.window, sink=s, rows=rows)
+
+
+def cpu_cores():
+    try:
+        aff = len(os.sched_getaffinity(0))
+    except AttributeError:
+        aff = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        blas = aff
+    return min(aff, blas), aff, blas
+
+
+def run_cpu_baseline(wl, rows_n, steps=1):
+    O, host, rows = oracle_sample(wl, rows_n)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle_step(O, host, rows, wl)
+    dt = time.perf_counter() - t0
+    used, aff, blas = cpu_cores()
+    return {"value": len(rows) * steps / dt, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": "%d query rows of %s (all four steps, float64 NumPy), %d step(s), %.1f s; "
+                      "affinity %d cores, BLAS threads %d" % (len(rows), wl.name, steps, dt, aff,
+                                                              blas)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas; control plane only)
+# ---------------------------------------------------------------------------
+
+def dist_init(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+class Step:
+    """Preallocated buffers and the four C-ABI calls of one forward step."""
+
+    def __init__(self, inp, wl):
+        self.inp, self.wl = inp, wl
+        T, H = inp.total_tokens, wl.num_heads
+        nb = hs.nbmax(inp.max_seqlen, wl.block_size)
+        dev = inp.q.device
+        f32 = torch.float32
+        self.lse1 = torch.empty((T, H), device=dev, dtype=f32)
+        self.bs = torch.empty((T, nb), device=dev, dtype=f32)
+        self.idx = torch.empty((T, wl.topk), device=dev, dtype=torch.int32)
+        self.out = torch.empty((T, H, wl.dv), device=dev, dtype=inp.q.dtype)
+        self.lse = torch.empty((T, H), device=dev, dtype=f32)
+        self.wout = torch.empty_like(self.out)
+        self.wlse = torch.empty_like(self.lse)
+        need = hs.workspace_size(hs.HS_OP_BLOCK_SCORE, T, len(wl.docs()), inp.max_seqlen, H,
+                                 wl.dk, wl.dv, inp.q.dtype, wl.block_size)
+        self.ws = torch.empty(max(need, 1), device=dev, dtype=torch.uint8)
+
+    def score(self):
+        i, w = self.inp, self.wl
+        hs.hs_block_score(i.q, i.k, i.cu_seqlens, i.max_seqlen, w.block_size, out_lse=self.lse1,
+                          out_block_score=self.bs, workspace=self.ws)
+
+    def select(self):
+        i, w = self.inp, self.wl
+        hs.hs_select_topk(self.bs, i.cu_seqlens, i.max_seqlen, w.block_size, w.topk,
+                          out_idx=self.idx)
+
+    def sparse(self):
+        i, w = self.inp, self.wl
+        hs.hs_sparse_mqa_fwd(i.q, i.k, i.v, self.idx, i.cu_seqlens, i.max_seqlen, w.block_size,
+                             i.sink, out=self.out, lse=self.lse)
+
+    def swa(self):
+        i, w = self.inp, self.wl
+        hs.hs_swa_mqa_fwd(i.q, i.k, i.v, i.cu_seqlens, i.max_seqlen, w.window, i.sink,
+                          out=self.wout, lse=self.wlse)
+
+    PHASES = ("score", "select", "sparse", "swa")
+
+    def run(self, events=None):
+        for n, ph in enumerate(self.PHASES):
+            if events is not None:
+                events[n].record()
+            getattr(self, ph)()
+        if events is not None:
+            events[len(self.PHASES)].record()
+
+
+def run_ours(args, wl, world, rank):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = synth.make_inputs(wl.total_tokens, wl.num_heads, wl.dk, wl.dv, dtype=wl.dtype, seed=rank,
+                            device=dev, doc_lengths=wl.docs())
+    step = Step(inp, wl)
+    flush = torch.empty(512 * 1024 * 1024, device=dev, dtype=torch.uint8)
+    for _ in range(max(3, args.warmup)):
+        step.run()
+    torch.cuda.synchronize()
+    hs.poll_status(dev)
+    cu = inp.cu_seqlens.cpu().tolist()
+
+    nph = len(Step.PHASES)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    for s in range(args.steps):
+        flush.fill_(s & 0xff)  # evict L2 between steps (outside the events)
+        step.run(evs[s])
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    hs.poll_status(dev)
+
+    per_phase = [[evs[s][p].elapsed_time(evs[s][p + 1]) for s in range(args.steps)]
+                 for p in range(nph)]
+    step_ms = [sum(per_phase[p][s] for p in range(nph)) for s in range(args.steps)]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    tokens = wl.total_tokens * world
+    value = tokens / (ms_per_step / 1e3)
+
+    pk = peaks()
+    H = wl.num_heads
+    flops = {
+        "score": 2.0 * H * wl.dk * causal_pairs(wl.docs()),
+        "sparse": 2.0 * H * (wl.dk + wl.dv) * sparse_pairs(step.idx, cu, wl.block_size),
+        "swa": 2.0 * H * (wl.dk + wl.dv) * window_pairs(wl.docs(), wl.window),
+    }
+    nb = hs.nbmax(inp.max_seqlen, wl.block_size)
+    sel_bytes = 4.0 * sum(((n - 1) // wl.block_size + 1) * n for n in wl.docs()) + 4.0 * wl.total_tokens * wl.topk
+    avg = {ph: statistics.mean(per_phase[p]) for p, ph in enumerate(Step.PHASES)}
+    kernels = {}
+    for ph in ("score", "sparse", "swa"):
+        tf = flops[ph] / (avg[ph] / 1e3) / 1e12
+        kernels[ph] = {"ms": avg[ph], "tflops": tf, "frac_of_bf16_peak": tf / pk["bf16_tflops"],
+                       "algorithmic_flops": flops[ph],
+                       "path": "tcgen05" if hs.path(
+                           {"score": 0, "sparse": 2, "swa": 3}[ph], wl.dtype, H, wl.dk, wl.dv,
+                           wl.block_size) == hs.HS_PATH_TCGEN05 else "simt"}
+    sel_gbs = sel_bytes / (avg["select"] / 1e3) / 1e9
+    kernels["select"] = {"ms": avg["select"], "gbs": sel_gbs, "frac_of_hbm": sel_gbs / pk["hbm_gbs"],
+                         "algorithmic_bytes": sel_bytes, "path": "simt"}
+    dom = max(("score", "sparse", "swa"), key=lambda ph: avg[ph])
+    roof = {"bound": "tensor", "achieved": kernels[dom]["tflops"], "peak": pk["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": kernels[dom]["tflops"] / pk["bf16_tflops"],
+            "traffic": None, "kernel": dom,
+            "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % pk["source"]}
+    contraction_tflops = (flops["score"] + flops["sparse"] + flops["swa"]) / (
+        (avg["score"] + avg["sparse"] + avg["swa"]) / 1e3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(inp, wl, step, max(3, min(args.steps, 10)), world)
+
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded N(0,1) q/k/v/sink, torch generator on device)",
+        "config": {"workload": wl.name, "tokens_per_gpu": wl.total_tokens, "num_heads": H,
+                   "dk": wl.dk, "dv": wl.dv, "block_size": wl.block_size, "topk": wl.topk,
+                   "window": wl.window, "docs": len(wl.docs()), "parallelism": "replicas x%d" % world,
+                   "l2": "flushed between steps (512 MiB write outside the timed events)",
+                   "step": "block_score + select_topk + sparse_mqa + swa_mqa"},
+        "roofline": roof,
+        "kernels": kernels,
+        "score_select_sparse_tokens_per_s": tokens / ((avg["score"] + avg["select"] + avg["sparse"]) / 1e3),
+        "contraction_tflops": contraction_tflops,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    return res
+
+
+def run_e2e(inp, wl, step, steps, world):
+    """Same metric through the public API with host buffers: every step copies
+    the inputs from pinned host memory, runs the four calls and copies the
+    outputs back; all inside the timed region."""
+    dev = inp.q.device
+    hq = inp.q.cpu().pin_memory()
+    hk = inp.k.cpu().pin_memory()
+    hv = inp.v.cpu().pin_memory()
+    hsink = inp.sink.cpu().pin_memory()
+    hcu = inp.cu_seqlens.cpu().pin_memory()
+    outs = [step.out, step.lse, step.wout, step.wlse, step.idx]
+    houts = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsink, hcu))
+    d2h = sum(t.numel() * t.element_size() for t in houts)
+
+    def one():
+        inp.q.copy_(hq, non_blocking=True)
+        inp.k.copy_(hk, non_blocking=True)
+        inp.v.copy_(hv, non_blocking=True)
+        inp.sink.copy_(hsink, non_blocking=True)
+        inp.cu_seqlens.copy_(hcu, non_blocking=True)
+        step.run()
+        for o, h in zip(outs, houts):
+            h.copy_(o, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world) / steps
+    return {"value": wl.total_tokens * world / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle on host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args, wl):
+    O, host, rows = oracle_sample(wl, args.cpu_rows)
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_step(O, host, rows[:2], wl)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(O, host, rows, wl)
+    dt = time.perf_counter() - t0
+    value = len(rows) * args.steps / dt
+    used, aff, blas = cpu_cores()
+    cb = {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+          "sample": "%d query rows of %s per step (all four steps, float64 NumPy); affinity %d "
+                    "cores, BLAS threads %d" % (len(rows), wl.name, aff, blas)}
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1), CPU generator)",
+            "config": {"workload": wl.name, "sample_rows_per_step": int(len(rows))},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    wl = workloads.ALL[args.workload]
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        if args.steps > 3:  # keep the CPU arm within minutes: fewer rows per step
+            args.cpu_rows = max(8, args.cpu_rows * 3 // args.steps)
+        print(json.dumps(run_reference(args, wl)), flush=True)
+        return 0
+    world, rank, local = dist_init(args)
+    res = run_ours(args, wl, world, rank)
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            res["cpu_baseline"] = run_cpu_baseline(wl, args.cpu_rows)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,328 @@
+// Host side of the libhs C ABI: argument validation, kernel choice, the
+// device status word and error reporting.  See include/hs.h for the contract
+// of every entry point.
+
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "hs.h"
+#include "hs_internal.h"
+
+namespace {
+
+// Device-side status word: kernels record the first device-detected problem
+// here (one copy per device that loads the library).
+__device__ int g_device_status;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices];
+std::mutex g_status_mu;
+
+std::atomic<int> g_force_simt{0};
+std::atomic<long long> g_wait_limit{0};
+
+thread_local char g_last_error[512];
+
+hs_status fail(hs_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+hs_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(HS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Address of the status word on the current device (looked up once per
+// device with that device current).
+hs_status status_ptr(int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(HS_ERR_UNSUPPORTED, "device id %d", dev);
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_status);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_status_ptr[dev];
+  return HS_OK;
+}
+
+bool valid_block(int b) { return b == 16 || b == 32 || b == 64 || b == 128; }
+
+int nbmax_of(int max_seqlen, int block_size) {
+  return (max_seqlen + block_size - 1) / block_size;
+}
+
+constexpr int kMaxHeads = 128;
+constexpr int kMaxDim = 1024;
+
+// Checks shared by the calls that read q and k; fills p (status excluded).
+hs_status check_problem(hs::Problem& p, const void* q, int64_t qrs, int64_t qhs, const void* k,
+                        int64_t krs, const int32_t* cu, int num_docs, int total_tokens,
+                        int max_seqlen, int num_heads, int dk, int dv, hs_dtype dtype,
+                        float scale) {
+  if (total_tokens < 0) return fail(HS_ERR_INVALID_ARG, "total_tokens < 0");
+  if (num_docs < 0) return fail(HS_ERR_INVALID_ARG, "num_docs < 0");
+  if (total_tokens > 0 && num_docs < 1)
+    return fail(HS_ERR_INVALID_ARG, "num_docs must be >= 1 when total_tokens > 0");
+  if (total_tokens > 0 && max_seqlen < 1)
+    return fail(HS_ERR_INVALID_ARG, "max_seqlen must be >= 1");
+  if (!cu) return fail(HS_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  if (!q || !k) return fail(HS_ERR_INVALID_ARG, "q or k is NULL");
+  if (dtype != HS_F32 && dtype != HS_BF16) return fail(HS_ERR_UNSUPPORTED, "dtype %d", (int)dtype);
+  if (num_heads < 1 || num_heads > kMaxHeads)
+    return fail(HS_ERR_UNSUPPORTED, "num_heads %d not in [1, %d]", num_heads, kMaxHeads);
+  if (dk < 1 || dk > kMaxDim) return fail(HS_ERR_UNSUPPORTED, "dk %d not in [1, %d]", dk, kMaxDim);
+  if (dv < 0 || dv > kMaxDim) return fail(HS_ERR_UNSUPPORTED, "dv %d not in [1, %d]", dv, kMaxDim);
+  if (qhs < dk) return fail(HS_ERR_INVALID_ARG, "q_head_stride %lld < dk", (long long)qhs);
+  if (qrs < (int64_t)num_heads * qhs)
+    return fail(HS_ERR_INVALID_ARG, "q_row_stride %lld < num_heads * q_head_stride", (long long)qrs);
+  if (krs < dk) return fail(HS_ERR_INVALID_ARG, "k_row_stride %lld < dk", (long long)krs);
+  if (!(isfinite(scale))) return fail(HS_ERR_INVALID_ARG, "softmax_scale is not finite");
+  p.q = q;
+  p.q_row_stride = qrs;
+  p.q_head_stride = qhs;
+  p.k = k;
+  p.k_row_stride = krs;
+  p.v = nullptr;
+  p.v_row_stride = 0;
+  p.cu_seqlens = cu;
+  p.num_docs = num_docs;
+  p.total_tokens = total_tokens;
+  p.max_seqlen = max_seqlen;
+  p.num_heads = num_heads;
+  p.dk = dk;
+  p.dv = dv;
+  p.dtype = dtype;
+  p.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)dk);
+  p.status = nullptr;
+  return HS_OK;
+}
+
+hs_status launched(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return HS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hs_version(void) { return 100; }
+
+const char* hs_status_string(hs_status s) {
+  switch (s) {
+    case HS_OK: return "HS_OK";
+    case HS_ERR_INVALID_ARG: return "HS_ERR_INVALID_ARG";
+    case HS_ERR_UNSUPPORTED: return "HS_ERR_UNSUPPORTED";
+    case HS_ERR_CUDA: return "HS_ERR_CUDA";
+    case HS_ERR_INVALID_INDEX: return "HS_ERR_INVALID_INDEX";
+    case HS_ERR_TIMEOUT: return "HS_ERR_TIMEOUT";
+    case HS_ERR_WORKSPACE: return "HS_ERR_WORKSPACE";
+  }
+  return "HS_ERR_UNKNOWN";
+}
+
+const char* hs_last_error(void) { return g_last_error; }
+
+void hs_set_force_simt(int on) { g_force_simt.store(on ? 1 : 0); }
+
+void hs_set_wait_limit(long long iterations) { g_wait_limit.store(iterations > 0 ? iterations : 0); }
+
+int hs_path(int op, hs_dtype dtype, int num_heads, int dk, int dv, int block_size) {
+  if (dtype != HS_F32 && dtype != HS_BF16) return -1;
+  switch (op) {
+    case HS_OP_SELECT_TOPK: return HS_PATH_SIMT;
+    case HS_OP_BLOCK_SCORE:
+      if (dtype == HS_BF16 && !g_force_simt.load() &&
+          hs::tc_block_score_supported(num_heads, dk, block_size, 0))
+        return HS_PATH_TCGEN05;
+      return HS_PATH_SIMT;
+    case HS_OP_SPARSE_MQA:
+    case HS_OP_SWA_MQA:
+      if (dtype == HS_BF16 && !g_force_simt.load() &&
+          hs::tc_attention_supported(num_heads, dk, dv, block_size, op == HS_OP_SPARSE_MQA))
+        return HS_PATH_TCGEN05;
+      return HS_PATH_SIMT;
+  }
+  return -1;
+}
+
+size_t hs_workspace_size(int op, int total_tokens, int num_docs, int max_seqlen, int num_heads,
+                         int dk, int dv, hs_dtype dtype, int block_size) {
+  (void)dv;
+  if (op != HS_OP_BLOCK_SCORE || total_tokens <= 0 || !valid_block(block_size)) return 0;
+  const int nbmax = nbmax_of(max_seqlen, block_size);
+  if (dtype == HS_BF16 && !g_force_simt.load() &&
+      hs::tc_block_score_supported(num_heads, dk, block_size, nbmax))
+    return hs::tc_block_score_workspace(total_tokens, num_docs, num_heads, nbmax);
+  return 0;
+}
+
+hs_status hs_poll_status(hs_stream_t stream) {
+  int* st = nullptr;
+  hs_status r = status_ptr(&st);
+  if (r != HS_OK) return r;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int host = 0;
+  e = cudaMemcpyFromSymbol(&host, g_device_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read status");
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clear status");
+  if (host != 0)
+    return fail((hs_status)host, "device reported %s", hs_status_string((hs_status)host));
+  return HS_OK;
+}
+
+hs_status hs_block_score(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                         const void* k, int64_t k_row_stride, const int32_t* cu_seqlens,
+                         int num_docs, int total_tokens, int max_seqlen, int num_heads, int dk,
+                         hs_dtype dtype, float softmax_scale, int block_size, float* lse,
+                         float* block_score, int nb_stride, float* block_lse, void* workspace,
+                         size_t workspace_bytes, hs_stream_t stream) {
+  hs::ScoreArgs a{};
+  hs_status r = check_problem(a.p, q, q_row_stride, q_head_stride, k, k_row_stride, cu_seqlens,
+                              num_docs, total_tokens, max_seqlen, num_heads, dk, 0, dtype,
+                              softmax_scale);
+  if (r != HS_OK) return r;
+  if (!valid_block(block_size))
+    return fail(HS_ERR_UNSUPPORTED, "block_size %d not in {16, 32, 64, 128}", block_size);
+  if (!lse || !block_score) return fail(HS_ERR_INVALID_ARG, "lse or block_score is NULL");
+  if (total_tokens == 0) return HS_OK;
+  const int nbmax = nbmax_of(max_seqlen, block_size);
+  if (nb_stride < nbmax)
+    return fail(HS_ERR_INVALID_ARG, "nb_stride %d < ceil(max_seqlen / block_size) = %d", nb_stride,
+                nbmax);
+  a.block_size = block_size;
+  a.nbmax = nbmax;
+  a.nb_stride = nb_stride;
+  a.lse = lse;
+  a.block_score = block_score;
+  a.block_lse = block_lse;
+  a.workspace = workspace;
+  a.workspace_bytes = workspace_bytes;
+  r = status_ptr(&a.p.status);
+  if (r != HS_OK) return r;
+  const bool tc = dtype == HS_BF16 && !g_force_simt.load() &&
+                  hs::tc_block_score_supported(num_heads, dk, block_size, nbmax);
+  if (tc) {
+    const size_t need = hs::tc_block_score_workspace(total_tokens, num_docs, num_heads, nbmax);
+    if (need > 0 && (!workspace || workspace_bytes < need))
+      return fail(HS_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                  workspace ? workspace_bytes : (size_t)0);
+    return launched(hs::launch_tc_block_score(a, g_wait_limit.load(), stream), "tc block score");
+  }
+  int dev = 0, optin = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (hs::simt_block_score_smem(num_heads, dk, nbmax) > (size_t)optin)
+    return fail(HS_ERR_UNSUPPORTED, "num_heads * dk + blocks too large for the CUDA-core kernel");
+  return launched(hs::launch_simt_block_score(a, stream), "simt block score");
+}
+
+hs_status hs_select_topk(const float* block_score, int nb_stride, const int32_t* cu_seqlens,
+                         int num_docs, int total_tokens, int max_seqlen, int block_size, int topk,
+                         int32_t* idx, hs_stream_t stream) {
+  if (total_tokens < 0 || num_docs < 0) return fail(HS_ERR_INVALID_ARG, "negative size");
+  if (total_tokens > 0 && (num_docs < 1 || max_seqlen < 1))
+    return fail(HS_ERR_INVALID_ARG, "num_docs and max_seqlen must be >= 1");
+  if (!block_score || !cu_seqlens || !idx) return fail(HS_ERR_INVALID_ARG, "NULL pointer");
+  if (!valid_block(block_size))
+    return fail(HS_ERR_UNSUPPORTED, "block_size %d not in {16, 32, 64, 128}", block_size);
+  if (topk < 1 || topk > 256) return fail(HS_ERR_UNSUPPORTED, "topk %d not in [1, 256]", topk);
+  if (total_tokens == 0) return HS_OK;
+  const int nbmax = nbmax_of(max_seqlen, block_size);
+  if (nb_stride < nbmax)
+    return fail(HS_ERR_INVALID_ARG, "nb_stride %d < ceil(max_seqlen / block_size) = %d", nb_stride,
+                nbmax);
+  int* st = nullptr;
+  hs_status r = status_ptr(&st);
+  if (r != HS_OK) return r;
+  return launched(hs::launch_select_topk(block_score, nb_stride, cu_seqlens, num_docs,
+                                         total_tokens, max_seqlen, block_size, topk, idx, st,
+                                         stream),
+                  "select topk");
+}
+
+static hs_status attention_common(hs::AttnArgs& a, bool sparse, const void* q, int64_t qrs,
+                                  int64_t qhs, const void* k, int64_t krs, const void* v,
+                                  int64_t vrs, const int32_t* cu, int num_docs, int total_tokens,
+                                  int max_seqlen, int num_heads, int dk, int dv, hs_dtype dtype,
+                                  float scale, const float* sink, void* out, float* lse,
+                                  hs_stream_t stream) {
+  hs_status r = check_problem(a.p, q, qrs, qhs, k, krs, cu, num_docs, total_tokens, max_seqlen,
+                              num_heads, dk, dv, dtype, scale);
+  if (r != HS_OK) return r;
+  if (dv < 1) return fail(HS_ERR_UNSUPPORTED, "dv must be >= 1");
+  if (!v) return fail(HS_ERR_INVALID_ARG, "v is NULL");
+  if (vrs < dv) return fail(HS_ERR_INVALID_ARG, "v_row_stride %lld < dv", (long long)vrs);
+  if (!out || !lse) return fail(HS_ERR_INVALID_ARG, "out or lse is NULL");
+  a.p.v = v;
+  a.p.v_row_stride = vrs;
+  a.sink = sink;
+  a.out = out;
+  a.lse = lse;
+  if (total_tokens == 0) return HS_OK;
+  r = status_ptr(&a.p.status);
+  if (r != HS_OK) return r;
+  const bool tc = dtype == HS_BF16 && !g_force_simt.load() &&
+                  hs::tc_attention_supported(num_heads, dk, dv, a.block_size, sparse);
+  if (tc) return launched(hs::launch_tc_attention(a, sparse, g_wait_limit.load(), stream),
+                          sparse ? "tc sparse attention" : "tc swa attention");
+  return launched(hs::launch_simt_attention(a, sparse, stream),
+                  sparse ? "simt sparse attention" : "simt swa attention");
+}
+
+hs_status hs_sparse_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                            const void* k, int64_t k_row_stride, const void* v,
+                            int64_t v_row_stride, const int32_t* cu_seqlens, int num_docs,
+                            int total_tokens, int max_seqlen, int num_heads, int dk, int dv,
+                            hs_dtype dtype, float softmax_scale, const int32_t* idx, int topk,
+                            int block_size, const float* sink, void* out, float* lse,
+                            hs_stream_t stream) {
+  if (!valid_block(block_size))
+    return fail(HS_ERR_UNSUPPORTED, "block_size %d not in {16, 32, 64, 128}", block_size);
+  if (topk < 1 || topk > 256) return fail(HS_ERR_UNSUPPORTED, "topk %d not in [1, 256]", topk);
+  if (!idx) return fail(HS_ERR_INVALID_ARG, "idx is NULL");
+  hs::AttnArgs a{};
+  a.idx = idx;
+  a.topk = topk;
+  a.block_size = block_size;
+  a.window = 0;
+  return attention_common(a, true, q, q_row_stride, q_head_stride, k, k_row_stride, v,
+                          v_row_stride, cu_seqlens, num_docs, total_tokens, max_seqlen,
+                          num_heads, dk, dv, dtype, softmax_scale, sink, out, lse, stream);
+}
+
+hs_status hs_swa_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                         const void* k, int64_t k_row_stride, const void* v, int64_t v_row_stride,
+                         const int32_t* cu_seqlens, int num_docs, int total_tokens,
+                         int max_seqlen, int num_heads, int dk, int dv, hs_dtype dtype,
+                         float softmax_scale, int window, const float* sink, void* out,
+                         float* lse, hs_stream_t stream) {
+  if (window < 1) return fail(HS_ERR_INVALID_ARG, "window %d < 1", window);
+  hs::AttnArgs a{};
+  a.idx = nullptr;
+  a.topk = 0;
+  a.block_size = 64;  // block size plays no part in the window; any valid value
+  a.window = window;
+  return attention_common(a, false, q, q_row_stride, q_head_stride, k, k_row_stride, v,
+                          v_row_stride, cu_seqlens, num_docs, total_tokens, max_seqlen,
+                          num_heads, dk, dv, dtype, softmax_scale, sink, out, lse, stream);
+}
+
+}  // extern "C"

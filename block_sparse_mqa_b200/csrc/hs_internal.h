@@ -1,0 +1,66 @@
+// Internal declarations shared by the libhs translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hs.h"
+
+namespace hs {
+
+// Arguments common to the attention-style calls, after host validation.
+struct Problem {
+  const void* q;
+  int64_t q_row_stride, q_head_stride;
+  const void* k;
+  int64_t k_row_stride;
+  const void* v;
+  int64_t v_row_stride;
+  const int32_t* cu_seqlens;
+  int num_docs, total_tokens, max_seqlen;
+  int num_heads, dk, dv;
+  hs_dtype dtype;
+  float scale;  // resolved (> 0)
+  int* status;  // device status word of the current device
+};
+
+struct ScoreArgs {
+  Problem p;
+  int block_size, nbmax, nb_stride;
+  float* lse;
+  float* block_score;
+  float* block_lse;  // may be null
+  void* workspace;
+  size_t workspace_bytes;
+};
+
+struct AttnArgs {
+  Problem p;
+  const int32_t* idx;  // sparse only
+  int topk, block_size;
+  int window;          // swa only
+  const float* sink;   // may be null
+  void* out;
+  float* lse;
+};
+
+// Launchers; each returns cudaSuccess or the launch error.
+cudaError_t launch_simt_block_score(const ScoreArgs& a, cudaStream_t s);
+cudaError_t launch_select_topk(const float* block_score, int nb_stride, const int32_t* cu,
+                               int num_docs, int total_tokens, int max_seqlen, int block_size,
+                               int topk, int32_t* idx, int* status, cudaStream_t s);
+cudaError_t launch_simt_attention(const AttnArgs& a, bool sparse, cudaStream_t s);
+
+// Shared-memory bytes the CUDA-core block-score kernel needs (0 if it cannot run).
+size_t simt_block_score_smem(int num_heads, int dk, int nbmax);
+
+// tcgen05 kernels (bf16).  *_supported() decides eligibility on the host.
+bool tc_block_score_supported(int num_heads, int dk, int block_size, int nbmax);
+size_t tc_block_score_workspace(int total_tokens, int num_docs, int num_heads, int nbmax);
+cudaError_t launch_tc_block_score(const ScoreArgs& a, long long wait_limit, cudaStream_t s);
+
+bool tc_attention_supported(int num_heads, int dk, int dv, int block_size, bool sparse);
+cudaError_t launch_tc_attention(const AttnArgs& a, bool sparse, long long wait_limit,
+                                cudaStream_t s);
+
+}  // namespace hs

@@ -1,0 +1,238 @@
+/*
+ * hs.h -- C ABI of libhs, the B200 (sm_100a) HySparse MQA forward path.
+ *
+ * The method: "HySparse MQA sparse attention (FA4 block scoring + SWA MQA +
+ * block-sparse DSA gather)", PaddleFleet pull request 1470 ("Core" list and
+ * the Copilot per-file table), in the absorbed-MLA MQA layout of its
+ * "FlashMLA sparse kernel constraints" section: H query heads share ONE key
+ * head of width Dk (latent + RoPE) and one value head of width Dv.
+ *
+ * Four calls form the forward path, in this order:
+ *   hs_block_score     causal QK^T pass -> per-head row LSE, per-head block
+ *                      LSE (optional) and head-summed block score
+ *   hs_select_topk     per-query top-k key blocks inside its document
+ *   hs_sparse_mqa_fwd  softmax attention over the selected blocks + sink
+ *   hs_swa_mqa_fwd     sliding-window attention + sink (Dk != Dv allowed)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Pointers named q, k, v, out, lse, block_score, block_lse, idx, sink and
+ * cu_seqlens are DEVICE pointers.  Element strides are in elements, not
+ * bytes; the innermost dimension of every tensor is contiguous.
+ *
+ *   q      [T, H, Dk]  row (token) stride q_row_stride, head stride
+ *                      q_head_stride.
+ *   k      [T, Dk]     row stride k_row_stride.
+ *   v      [T, Dv]     row stride v_row_stride; may alias k (for example
+ *                      v = k with Dv < Dk reads the first Dv columns, the
+ *                      absorbed-MLA latent region).
+ *   cu_seqlens [num_docs + 1] int32: packed documents; cu_seqlens[0] = 0,
+ *                      non-decreasing, cu_seqlens[num_docs] = T.  Document d
+ *                      is tokens [cu_seqlens[d], cu_seqlens[d+1]).  No
+ *                      attention, block or window crosses a document end.
+ *   max_seqlen         host-side upper bound of every document's length; it
+ *                      sizes grids and the block count NBmax =
+ *                      ceil(max_seqlen / block_size).
+ *   dtype              HS_BF16 or HS_F32 for q, k, v and out (all the same).
+ *                      Accumulation is fp32 in every case.
+ *   softmax_scale      logits are s = softmax_scale * <q, k>; a value <= 0
+ *                      selects Dk^-1/2 (the default sm_scale of the SWA
+ *                      wrapper, per-file table entry "swa_attn.py").
+ *   stream             a cudaStream_t (NULL = legacy default stream).  All
+ *                      calls are asynchronous on it.
+ *
+ * Blocks.  Key blocks of size B are laid on each document separately from
+ * its first token (the per-document block_bos of the block-score PyLayer in
+ * the review of PaddleFleet pull request 1453); the last block of a
+ * document may be partial.  Block ids are document-local.  For a query t
+ * of document [bos, eos), its own block is bq(t) = (t - bos) / B.
+ *
+ * Ownership.  The caller owns every buffer, its allocation and lifetime.
+ * The library never allocates, frees or synchronises inside these four
+ * calls; any scratch it needs is the caller's `workspace` argument.
+ *
+ * Errors.  Every call validates its host-visible arguments before any
+ * launch and returns a non-zero hs_status without touching the GPU when
+ * they are wrong.  Device-detected problems (a malformed cu_seqlens, an
+ * out-of-range block id, a pipeline wait that ran out of its iteration
+ * limit) never trap: the kernel records a status word, skips the bad work
+ * and exits; hs_poll_status() returns it.  hs_last_error() describes the
+ * most recent host-side failure of the calling thread.
+ */
+#ifndef HS_H_
+#define HS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hs_stream_t; /* == cudaStream_t */
+
+typedef enum hs_status {
+  HS_OK = 0,
+  HS_ERR_INVALID_ARG = 1,   /* bad pointer, size, stride or cu_seqlens     */
+  HS_ERR_UNSUPPORTED = 2,   /* valid but not implemented (dtype, dims)     */
+  HS_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed        */
+  HS_ERR_INVALID_INDEX = 4, /* device: a block id outside [-1, bq]         */
+  HS_ERR_TIMEOUT = 5,       /* device: a bounded pipeline wait ran out     */
+  HS_ERR_WORKSPACE = 6      /* workspace missing or smaller than required  */
+} hs_status;
+
+typedef enum hs_dtype { HS_F32 = 0, HS_BF16 = 1 } hs_dtype;
+
+/* Operation ids for hs_path() and hs_workspace_size(). */
+typedef enum hs_op {
+  HS_OP_BLOCK_SCORE = 0,
+  HS_OP_SELECT_TOPK = 1,
+  HS_OP_SPARSE_MQA = 2,
+  HS_OP_SWA_MQA = 3
+} hs_op;
+
+/* Kernel family a call will use, as returned by hs_path(). */
+typedef enum hs_kernel_path {
+  HS_PATH_SIMT = 0,   /* CUDA-core kernel: fp32 inputs, unusual shapes    */
+  HS_PATH_TCGEN05 = 1 /* tcgen05 tensor-core kernel (TMEM accumulators)   */
+} hs_kernel_path;
+
+/*
+ * Step 1 -- causal block scoring.
+ * Source: "HySparse MQA sparse attention ...", PaddleFleet pull request
+ * 1470, "Core" list (FA4-fused block scoring) and per-file table
+ * (pipeline.py: the block score is recovered as exp(block_logit - lse)
+ * before top-k); review of pull request 1453 (per-document block_bos).
+ *
+ * For query t in document [bos, eos), head h, s_j = scale * <q[t,h], k[j]>
+ * over the causal keys j in [bos, t]:
+ *   lse[t,h]          = log sum_j exp(s_j)                 (no sink)
+ *   block_lse[t,h,b]  = log sum_{j in block b, j <= t} exp(s_j)
+ *   block_score[t,b]  = sum_h exp(block_lse[t,h,b] - lse[t,h])
+ * for b <= bq(t); for bq(t) < b < NBmax, block_score = 0 and block_lse =
+ * -inf.  Columns NBmax .. nb_stride-1 are not written.  Logs are natural.
+ *
+ *   lse          [T, H] fp32, output.
+ *   block_score  [T, nb_stride] fp32, output; nb_stride >= NBmax.
+ *   block_lse    [T, H, nb_stride] fp32, optional output (NULL = skip).
+ *   workspace    device scratch of at least
+ *                hs_workspace_size(HS_OP_BLOCK_SCORE, ...) bytes (may be
+ *                NULL when that size is 0).  Its contents on entry do not
+ *                matter; concurrent calls must not share one workspace.
+ *   block_size   16, 32, 64 or 128.
+ */
+hs_status hs_block_score(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                         const void* k, int64_t k_row_stride,
+                         const int32_t* cu_seqlens, int num_docs, int total_tokens,
+                         int max_seqlen, int num_heads, int dk, hs_dtype dtype,
+                         float softmax_scale, int block_size,
+                         float* lse, float* block_score, int nb_stride, float* block_lse,
+                         void* workspace, size_t workspace_bytes, hs_stream_t stream);
+
+/*
+ * Step 2 -- per-query top-k block selection.
+ * Source: per-file table of pull request 1470 (pipeline.py: top-k block
+ * selection over the recovered block scores).  Rule: candidates are blocks
+ * 0..bq(t) of the query's document; the own block bq(t) and the first
+ * block 0 are always selected and count toward topk; when bq(t) + 1 <=
+ * topk all candidates are selected; otherwise the remaining slots go to
+ * the highest block_score values, an exact fp32 tie going to the lower
+ * block id.
+ *
+ *   block_score  [T, nb_stride] fp32 (as written by hs_block_score); only
+ *                columns 0..bq(t) of row t are read.
+ *   idx          [T, topk] int32 output: document-local block ids in
+ *                ascending order, unused slots = -1.
+ *   topk         1..256.  topk = 1 selects only the own block (the first
+ *                block is then not forced).
+ */
+hs_status hs_select_topk(const float* block_score, int nb_stride,
+                         const int32_t* cu_seqlens, int num_docs, int total_tokens,
+                         int max_seqlen, int block_size, int topk, int32_t* idx,
+                         hs_stream_t stream);
+
+/*
+ * Step 3 -- block-sparse MQA attention with a per-head sink.
+ * Source: pull request 1470, "Core" list (block-sparse DSA gather with a
+ * learnable per-head attn_sink) and "FlashMLA sparse kernel constraints";
+ * the sink is a softmax offset ("Support attn sink in fa3", pull request
+ * 1415, dense-path review thread): a logit in the denominator only.
+ *
+ * Keys of query t: S_t = union over the ids b >= 0 in idx[t] of the keys of
+ * block b that are <= t.  With s_j = scale * <q[t,h], k[j]>:
+ *   lse[t,h] = log(exp(sink[h]) + sum_{j in S_t} exp(s_j))
+ *   out[t,h] = sum_{j in S_t} exp(s_j - lse[t,h]) * v[j]
+ * sink is in the scaled logit space (not multiplied by softmax_scale).
+ *
+ *   idx    [T, topk] int32: ascending distinct ids in [0, bq(t)], then -1
+ *          padding (the output of hs_select_topk).  An id outside
+ *          [-1, bq(t)] is skipped and reported as HS_ERR_INVALID_INDEX.
+ *   sink   [H] fp32 or NULL (NULL = no sink, i.e. -inf).
+ *   out    [T, H, Dv] of `dtype`, contiguous, output.
+ *   lse    [T, H] fp32, output.
+ */
+hs_status hs_sparse_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                            const void* k, int64_t k_row_stride,
+                            const void* v, int64_t v_row_stride,
+                            const int32_t* cu_seqlens, int num_docs, int total_tokens,
+                            int max_seqlen, int num_heads, int dk, int dv, hs_dtype dtype,
+                            float softmax_scale, const int32_t* idx, int topk,
+                            int block_size, const float* sink,
+                            void* out, float* lse, hs_stream_t stream);
+
+/*
+ * Step 4 -- sliding-window MQA attention with a per-head sink.
+ * Source: pull request 1470, "Core" list (SWA sliding-window MQA) and
+ * per-file table (windowed_mqa_attn*.py: Dk != Dv, optional attn_sink);
+ * review of pull request 1453 (per-row bos/eos key ranges).
+ *
+ * Keys of query t: the `window` keys ending at t, clipped at its document
+ * start: j in [max(bos, t - window + 1), t].  Same lse/out/sink formulas
+ * as hs_sparse_mqa_fwd.  window >= 1.
+ */
+hs_status hs_swa_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                         const void* k, int64_t k_row_stride,
+                         const void* v, int64_t v_row_stride,
+                         const int32_t* cu_seqlens, int num_docs, int total_tokens,
+                         int max_seqlen, int num_heads, int dk, int dv, hs_dtype dtype,
+                         float softmax_scale, int window, const float* sink,
+                         void* out, float* lse, hs_stream_t stream);
+
+/* ---------------------------------------------------------------- helpers */
+
+/* Bytes of `workspace` that op needs for these sizes (0 = none).  Only
+ * HS_OP_BLOCK_SCORE uses a workspace. */
+size_t hs_workspace_size(int op, int total_tokens, int num_docs, int max_seqlen,
+                         int num_heads, int dk, int dv, hs_dtype dtype, int block_size);
+
+/* Which kernel family op would run for these parameters (hs_kernel_path),
+ * or -1 when the parameters are unsupported. */
+int hs_path(int op, hs_dtype dtype, int num_heads, int dk, int dv, int block_size);
+
+/* Synchronises `stream`, then returns and clears the device-side status
+ * word (HS_OK when no kernel recorded a problem).  This is the only call
+ * that waits for the GPU. */
+hs_status hs_poll_status(hs_stream_t stream);
+
+/* Testing aid: when on != 0 every call uses the CUDA-core kernels even
+ * where a tensor-core kernel exists.  Process-wide; not for production. */
+void hs_set_force_simt(int on);
+
+/* Testing aid: overrides the iteration limit of the tensor-core kernels'
+ * pipeline waits (0 restores the default).  A tiny limit makes the waits
+ * give up early and report HS_ERR_TIMEOUT instead of computing. */
+void hs_set_wait_limit(long long iterations);
+
+const char* hs_status_string(hs_status status);
+
+/* Message of the calling thread's most recent failed call ("" if none). */
+const char* hs_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int hs_version(void);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* HS_H_ */

@@ -1,0 +1,118 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol
+include/hs.h declares, and rejects bad arguments on the host before any CUDA
+call (validation comes first, so these calls never touch a device)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_mqa_b200 import hs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "hs.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hs_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = hs.lib()
+    names = _declared()
+    assert "hs_block_score" in names and "hs_swa_mqa_fwd" in names
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(hs.EXPORTS)
+
+
+def test_helpers():
+    L = hs.lib()
+    assert L.hs_version() >= 100
+    assert L.hs_status_string(hs.HS_ERR_TIMEOUT) == b"HS_ERR_TIMEOUT"
+    assert hs.path(hs.HS_OP_SELECT_TOPK, __import__("torch").float32, 4, 64, 48, 16) == hs.HS_PATH_SIMT
+    assert L.hs_path(0, 7, 64, 576, 512, 64) == -1
+
+
+_I64 = ctypes.c_int64
+NULL = None
+
+
+def _score(**kw):
+    a = dict(q=1, qrs=64 * 576, qhs=576, k=1, krs=576, cu=1, nd=1, T=128, maxlen=128, H=64,
+             dk=576, dt=hs.HS_BF16, scale=0.0, B=64, lse=1, bs=1, nbs=2, blse=NULL, ws=NULL,
+             wsb=0)
+    a.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return hs.lib().hs_block_score(v(a["q"]), a["qrs"], a["qhs"], v(a["k"]), a["krs"], v(a["cu"]),
+                                   a["nd"], a["T"], a["maxlen"], a["H"], a["dk"], a["dt"],
+                                   a["scale"], a["B"], v(a["lse"]), v(a["bs"]), a["nbs"],
+                                   v(a["blse"]), v(a["ws"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), hs.HS_ERR_INVALID_ARG),
+    (dict(cu=None), hs.HS_ERR_INVALID_ARG),
+    (dict(T=-1), hs.HS_ERR_INVALID_ARG),
+    (dict(nd=0), hs.HS_ERR_INVALID_ARG),
+    (dict(maxlen=0), hs.HS_ERR_INVALID_ARG),
+    (dict(H=0), hs.HS_ERR_UNSUPPORTED),
+    (dict(H=129), hs.HS_ERR_UNSUPPORTED),
+    (dict(dk=2048), hs.HS_ERR_UNSUPPORTED),
+    (dict(dt=5), hs.HS_ERR_UNSUPPORTED),
+    (dict(qhs=100), hs.HS_ERR_INVALID_ARG),
+    (dict(qrs=576), hs.HS_ERR_INVALID_ARG),
+    (dict(krs=5), hs.HS_ERR_INVALID_ARG),
+    (dict(B=48), hs.HS_ERR_UNSUPPORTED),
+    (dict(lse=None), hs.HS_ERR_INVALID_ARG),
+    (dict(nbs=1), hs.HS_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), hs.HS_ERR_INVALID_ARG),
+])
+def test_block_score_rejects_bad_arguments(kw, code):
+    assert _score(**kw) == code
+    assert hs.lib().hs_last_error()  # a message was recorded
+
+
+def test_empty_input_is_a_no_op():
+    # zero tokens: valid, nothing launched (no GPU needed)
+    assert _score(T=0, nd=0, maxlen=0) == hs.HS_OK
+
+
+def test_select_rejects_bad_arguments():
+    L = hs.lib()
+    p = ctypes.c_void_p(1)
+    assert L.hs_select_topk(p, 4, p, 1, 100, 100, 64, 0, p, None) == hs.HS_ERR_UNSUPPORTED
+    assert L.hs_select_topk(p, 4, p, 1, 100, 100, 64, 257, p, None) == hs.HS_ERR_UNSUPPORTED
+    assert L.hs_select_topk(p, 1, p, 1, 100, 100, 64, 4, p, None) == hs.HS_ERR_INVALID_ARG
+    assert L.hs_select_topk(None, 4, p, 1, 100, 100, 64, 4, p, None) == hs.HS_ERR_INVALID_ARG
+    assert L.hs_select_topk(p, 4, p, 1, 100, 100, 20, 4, p, None) == hs.HS_ERR_UNSUPPORTED
+
+
+def test_attention_rejects_bad_arguments():
+    L = hs.lib()
+    p = ctypes.c_void_p(1)
+    args = [p, 64 * 576, 576, p, 576, p, 512, p, 1, 100, 100, 64, 576, 512, hs.HS_BF16, 0.0]
+    # sparse: topk 0, NULL idx, bad block, bad v stride, NULL out
+    assert L.hs_sparse_mqa_fwd(*args, p, 0, 64, None, p, p, None) == hs.HS_ERR_UNSUPPORTED
+    assert L.hs_sparse_mqa_fwd(*args, None, 4, 64, None, p, p, None) == hs.HS_ERR_INVALID_ARG
+    assert L.hs_sparse_mqa_fwd(*args, p, 4, 8, None, p, p, None) == hs.HS_ERR_UNSUPPORTED
+    bad_v = list(args)
+    bad_v[6] = 100
+    assert L.hs_sparse_mqa_fwd(*bad_v, p, 4, 64, None, p, p, None) == hs.HS_ERR_INVALID_ARG
+    assert L.hs_sparse_mqa_fwd(*args, p, 4, 64, None, None, p, None) == hs.HS_ERR_INVALID_ARG
+    # swa: window 0, dv 0
+    assert L.hs_swa_mqa_fwd(*args, 0, None, p, p, None) == hs.HS_ERR_INVALID_ARG
+    no_dv = list(args)
+    no_dv[13] = 0
+    assert L.hs_swa_mqa_fwd(*no_dv, 16, None, p, p, None) == hs.HS_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(4, 2, 8)
+    k = torch.zeros(4, 8)
+    cu = torch.tensor([0, 4], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        hs.hs_block_score(q, k, cu, 4, 16)

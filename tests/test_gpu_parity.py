@@ -1,0 +1,207 @@
+"""GPU parity: every step of the CUDA path against the float64 CPU oracle on
+the same seeded inputs, through the C ABI (ctypes binding).
+
+Small cases compare every output element; the full-size workloads compare a
+seeded sample of query rows (the oracle computes those rows one by one).
+Tolerances are in tests/parity.py.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.hysparse as O
+from block_sparse_mqa_b200 import hs, synth, workloads
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _gpu_inputs(T, H, dk, dv, dtype, docs, seed=0, sink_std=1.0):
+    return synth.make_inputs(T, H, dk, dv, dtype=dtype, seed=seed, device=DEV, doc_lengths=docs,
+                             sink_std=sink_std)
+
+
+def _host(inp):
+    f = lambda t: t.detach().cpu().double().numpy()
+    return f(inp.q), f(inp.k), f(inp.v), f(inp.sink), inp.cu_seqlens.cpu().tolist()
+
+
+def _expect_path(op, inp, B):
+    return hs.path(op, inp.q.dtype, inp.q.shape[1], inp.q.shape[2], inp.v.shape[1], B)
+
+
+def run_and_check(inp, B, K, W, rows=None, sink=True, scale=0.0, v=None, check_paths=None):
+    """Run the four steps on the GPU and compare each against the oracle
+    (stage-isolated: the oracle's select/attention take the GPU's scores /
+    indices as inputs, and the end-to-end index sets are compared too)."""
+    q, k, vv, s, cu = _host(inp)
+    v_dev = inp.v if v is None else v
+    if v is not None:
+        vv = v.detach().cpu().double().numpy()
+    sink_dev = inp.sink if sink else None
+    sink_np = s if sink else None
+    T = inp.total_tokens
+    rr = np.arange(T) if rows is None else np.asarray(rows)
+    sc = None if scale == 0.0 else scale
+
+    lse1, bs, blse = hs.hs_block_score(inp.q, inp.k, inp.cu_seqlens, inp.max_seqlen, B, scale,
+                                       want_block_lse=rows is None)
+    idx = hs.hs_select_topk(bs, inp.cu_seqlens, inp.max_seqlen, B, K)
+    out, lse = hs.hs_sparse_mqa_fwd(inp.q, inp.k, v_dev, idx, inp.cu_seqlens, inp.max_seqlen, B,
+                                    sink_dev, scale)
+    wout, wlse = hs.hs_swa_mqa_fwd(inp.q, inp.k, v_dev, inp.cu_seqlens, inp.max_seqlen, W,
+                                   sink_dev, scale)
+    torch.cuda.synchronize()
+    hs.poll_status()
+
+    rows_t = torch.as_tensor(rr, device=DEV)
+    ref1 = O.block_score(q, k, cu, B, scale=sc, rows=rr)
+    nb = ref1["block_score"].shape[1]
+    P.check_lse(lse1[rows_t], ref1["lse"], "score lse")
+    P.check_scores(bs[rows_t], ref1["block_score"])
+    if blse is not None:
+        P.check_lse(blse[rows_t][:, :, :nb], ref1["block_lse"], "block_lse")
+    # select: bit-exact on the GPU's own scores, near-tie rule against the oracle's
+    bs_rows = bs[rows_t].double().cpu().numpy()
+    idx_rows = idx[rows_t].cpu().numpy()
+    ref_idx_same = O.select_topk(bs_rows, cu, B, K, rows=rr, total_tokens=T)
+    np.testing.assert_array_equal(idx_rows, ref_idx_same)
+    ref_idx = O.select_topk(ref1["block_score"], cu, B, K, rows=rr, total_tokens=T)
+    P.check_topk(idx_rows, ref_idx, ref1["block_score"], P.bq_rows(cu, rr, B), K)
+    # attention on the GPU's indices
+    ref3 = O.sparse_mqa_fwd(q, k, vv, idx_rows, cu, B, sink=sink_np, scale=sc, rows=rr)
+    P.check_out(out[rows_t], ref3["out"], "sparse out")
+    P.check_lse(lse[rows_t], ref3["lse"], "sparse lse")
+    ref4 = O.swa_mqa_fwd(q, k, vv, cu, W, sink=sink_np, scale=sc, rows=rr)
+    P.check_out(wout[rows_t], ref4["out"], "swa out")
+    P.check_lse(wlse[rows_t], ref4["lse"], "swa lse")
+    return {"idx": idx, "out": out, "lse": lse, "swa_out": wout, "swa_lse": wlse, "bs": bs,
+            "lse1": lse1}
+
+
+# ---------------------------------------------------------------------------
+# small cases, every element
+# ---------------------------------------------------------------------------
+
+def test_tiny_fp32_workload():
+    wl = workloads.TINY
+    inp = _gpu_inputs(wl.total_tokens, wl.num_heads, wl.dk, wl.dv, wl.dtype, wl.docs())
+    for op in (hs.HS_OP_BLOCK_SCORE, hs.HS_OP_SPARSE_MQA, hs.HS_OP_SWA_MQA):
+        assert _expect_path(op, inp, wl.block_size) == hs.HS_PATH_SIMT
+    run_and_check(inp, wl.block_size, wl.topk, wl.window)
+
+
+@pytest.mark.parametrize("docs", [[452], [130, 64, 1, 257], [63, 65, 200, 124]])
+def test_mla_shape_small_packed(docs):
+    T = sum(docs)
+    inp = _gpu_inputs(T, 64, 576, 512, torch.bfloat16, docs, seed=1)
+    run_and_check(inp, 64, 4, 100)
+
+
+@pytest.mark.parametrize("B,K,W", [(16, 3, 1), (32, 2, 700), (128, 5, 129), (64, 1, 64)])
+def test_block_window_variants(B, K, W):
+    docs = [300, 37, 180]
+    inp = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=2)
+    run_and_check(inp, B, K, W)
+
+
+def test_no_sink_and_large_sink():
+    docs = [200, 77]
+    inp = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=3)
+    run_and_check(inp, 64, 3, 90, sink=False)
+    inp.sink.fill_(8.0)
+    run_and_check(inp, 64, 3, 90, sink=True)
+
+
+def test_v_aliases_latent_part_of_k():
+    docs = [260]
+    inp = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=4)
+    v_alias = inp.k[:, :512]  # absorbed-MLA: value = latent region of the key row
+    assert v_alias.data_ptr() == inp.k.data_ptr()
+    run_and_check(inp, 64, 3, 128, v=v_alias)
+
+
+def test_strided_q_and_explicit_scale():
+    docs = [150, 90]
+    T = sum(docs)
+    base = _gpu_inputs(T, 64, 576, 512, torch.bfloat16, docs, seed=5)
+    big = torch.zeros((T, 66, 640), device=DEV, dtype=torch.bfloat16)
+    big[:, :64, :576] = base.q
+    base.q = big[:, :64, :576]
+    assert base.q.stride() == (66 * 640, 640, 1)
+    run_and_check(base, 64, 3, 70, scale=0.03)
+
+
+def test_other_head_counts_and_dims():
+    for H, dk, dv in ((4, 64, 48), (16, 192, 128), (64, 192, 128), (8, 40, 24)):
+        docs = [150, 61]
+        inp = _gpu_inputs(sum(docs), H, dk, dv, torch.bfloat16, docs, seed=6)
+        run_and_check(inp, 16, 4, 33)
+
+
+def test_force_simt_agrees_with_default_path():
+    docs = [333, 80]
+    inp = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=7)
+    a = hs.hs_forward(inp.q, inp.k, inp.v, inp.cu_seqlens, inp.max_seqlen, 64, 4, 100, inp.sink)
+    hs.set_force_simt(True)
+    try:
+        b = hs.hs_forward(inp.q, inp.k, inp.v, inp.cu_seqlens, inp.max_seqlen, 64, 4, 100, inp.sink)
+    finally:
+        hs.set_force_simt(False)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(a["block_score"].cpu(), b["block_score"].cpu(), rtol=2e-4, atol=1e-5)
+    P.check_lse(a["sparse_lse"], P.np64(b["sparse_lse"]))
+    P.check_out(a["swa_out"], P.np64(b["swa_out"]))
+
+
+# ---------------------------------------------------------------------------
+# device-detected errors
+# ---------------------------------------------------------------------------
+
+def test_invalid_index_reported():
+    docs = [200]
+    inp = _gpu_inputs(200, 64, 576, 512, torch.bfloat16, docs, seed=8)
+    idx = torch.full((200, 2), -1, device=DEV, dtype=torch.int32)
+    idx[:, 0] = torch.arange(200, device=DEV, dtype=torch.int32) // 64
+    idx[5, 1] = 3  # block 3 is in the future of token 5
+    hs.hs_sparse_mqa_fwd(inp.q, inp.k, inp.v, idx, inp.cu_seqlens, 200, 64, inp.sink)
+    with pytest.raises(hs.HSError) as e:
+        hs.poll_status()
+    assert e.value.status == hs.HS_ERR_INVALID_INDEX
+    hs.poll_status()  # cleared
+
+
+def test_malformed_cu_seqlens_reported():
+    inp = _gpu_inputs(128, 64, 576, 512, torch.bfloat16, [128], seed=9)
+    bad = torch.tensor([0, 100, 128], device=DEV, dtype=torch.int32)
+    # max_seqlen 64 is smaller than the first document: rows of it are skipped
+    lse, bs, _ = hs.hs_block_score(inp.q, inp.k, bad, 64, 64)
+    with pytest.raises(hs.HSError) as e:
+        hs.poll_status()
+    assert e.value.status == hs.HS_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, sampled rows
+# ---------------------------------------------------------------------------
+
+def _sampled(wl, per_doc, seed=0):
+    inp = _gpu_inputs(wl.total_tokens, wl.num_heads, wl.dk, wl.dv, wl.dtype, wl.docs(), seed=seed)
+    rows = synth.sample_rows(inp.cu_seqlens.cpu(), per_doc, seed)
+    return inp, rows
+
+
+def test_main_workload_sampled():
+    wl = workloads.MAIN
+    inp, rows = _sampled(wl, 48)
+    run_and_check(inp, wl.block_size, wl.topk, wl.window, rows=rows)
+
+
+@pytest.mark.slow
+def test_packed_workload_sampled():
+    wl = workloads.PACKED
+    inp, rows = _sampled(wl, 12)
+    run_and_check(inp, wl.block_size, wl.topk, wl.window, rows=rows)
