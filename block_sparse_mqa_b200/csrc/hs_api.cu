@@ -218,7 +218,8 @@ hs_status hs_block_score(const void* q, int64_t q_row_stride, int64_t q_head_str
   r = status_ptr(&a.p.status);
   if (r != HS_OK) return r;
   const bool tc = dtype == HS_BF16 && !g_force_simt.load() &&
-                  hs::tc_block_score_supported(num_heads, dk, block_size, nbmax);
+                  hs::tc_block_score_supported(num_heads, dk, block_size, nbmax) &&
+                  hs::tc_block_score_eligible(a);
   if (tc) {
     const size_t need = hs::tc_block_score_workspace(total_tokens, num_docs, num_heads, nbmax);
     if (need > 0 && (!workspace || workspace_bytes < need))
@@ -280,7 +281,8 @@ static hs_status attention_common(hs::AttnArgs& a, bool sparse, const void* q, i
   r = status_ptr(&a.p.status);
   if (r != HS_OK) return r;
   const bool tc = dtype == HS_BF16 && !g_force_simt.load() &&
-                  hs::tc_attention_supported(num_heads, dk, dv, a.block_size, sparse);
+                  hs::tc_attention_supported(num_heads, dk, dv, a.block_size, sparse) &&
+                  hs::tc_attention_eligible(a);
   if (tc) return launched(hs::launch_tc_attention(a, sparse, g_wait_limit.load(), stream),
                           sparse ? "tc sparse attention" : "tc swa attention");
   return launched(hs::launch_simt_attention(a, sparse, stream),

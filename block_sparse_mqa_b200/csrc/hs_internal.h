@@ -57,9 +57,11 @@ size_t simt_block_score_smem(int num_heads, int dk, int nbmax);
 // tcgen05 kernels (bf16).  *_supported() decides eligibility on the host.
 bool tc_block_score_supported(int num_heads, int dk, int block_size, int nbmax);
 size_t tc_block_score_workspace(int total_tokens, int num_docs, int num_heads, int nbmax);
+bool tc_block_score_eligible(const ScoreArgs& a);  // alignment / doc-count conditions
 cudaError_t launch_tc_block_score(const ScoreArgs& a, long long wait_limit, cudaStream_t s);
 
 bool tc_attention_supported(int num_heads, int dk, int dv, int block_size, bool sparse);
+bool tc_attention_eligible(const AttnArgs& a);  // alignment conditions
 cudaError_t launch_tc_attention(const AttnArgs& a, bool sparse, long long wait_limit,
                                 cudaStream_t s);
 

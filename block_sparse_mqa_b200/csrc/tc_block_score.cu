@@ -1,0 +1,538 @@
+// hs_block_score on tcgen05 tensor cores (bf16 in, fp32 accumulate).
+//
+// Definition ("HySparse MQA sparse attention ...", PaddleFleet pull request
+// 1470: "Core" list, FA4-fused block scoring; per-file table, pipeline.py:
+// block score = exp(block_logit - lse)): for query t, head h and block b <=
+// bq(t) of t's document, blockLSE = log sum_{j in block b, j <= t} exp(s_j),
+// LSE = log sum_{j <= t} exp(s_j), score[t, b] = sum_h exp(blockLSE - LSE).
+//
+// Design (one persistent CTA per SM, 6 warps):
+//  * A query tile is 128 rows = (128 / H) consecutive tokens x H heads of one
+//    document; q[T, H, Dk] rows are (token, head) pairs, so a tile is a
+//    plain 128-row slab.  The first min(Dk, 512) columns of the tile live in
+//    TMEM as the A operand (TS form: written by the softmax threads, one row
+//    each); any remaining 64-column chunk (the RoPE part of Dk = 576) is a
+//    128-byte-swizzled shared-memory tile loaded by TMA (SS form).
+//  * Keys stream in tiles of 128 (always a whole number of blocks, starting
+//    at the document's first token) as 64-column K chunks through an 8-deep
+//    TMA ring of 16 KB stages; each chunk feeds four M=128, N=128, K=16 MMAs
+//    into one of two S accumulators in TMEM (double buffering lets the MMA
+//    run one key tile ahead of the softmax).
+//  * Softmax warps (thread = row) read S (tcgen05.ld), compute per-block
+//    log-sum-exp in the log2 domain with the block's own max (no underflow
+//    for far-below-max blocks) and keep the running row max and sum.  Block
+//    values go to a per-CTA global workspace slot [NBmax][128] (coalesced,
+//    L2 resident).  At the end of the tile each row has its LSE; the head
+//    sum of exp2(blockLSE - LSE) is a 32-lane transpose-reduction per warp
+//    plus a fixed-order sum over the warps of a token (deterministic).
+//  * Warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner), warps 2-5
+//    = softmax / Q loader / epilogue.  Every wait is bounded; a timeout
+//    records HS_ERR_TIMEOUT, drains in-flight copies and MMAs, frees TMEM.
+
+#include <math.h>
+
+#include "hs_device.cuh"
+#include "hs_internal.h"
+#include "tc_common.cuh"
+#include "tc_host.h"
+
+namespace hs {
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 192;
+constexpr int kStages = 8;
+constexpr int kKeyTile = 128;
+constexpr int kStageBytes = kKeyTile * 64 * 2;  // 128 keys x 64 bf16
+constexpr int kMaxQhi = 2;                       // shared-memory Q chunks (Dk <= 640)
+constexpr int kMaxTmemQ = 8;                     // TMEM Q chunks (first 512 columns)
+constexpr int kMaxDocs = 1024;
+constexpr int kSCol = 256;                       // S buffers at TMEM columns 256, 384
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kLog2e = 1.44269504088896340736f;
+
+struct BSParams {
+  const int32_t* cu;
+  int num_docs, T, max_seqlen;
+  const __nv_bfloat16* q;
+  int64_t qrs, qhs;
+  int H, nck, nq_tmem, nq_smem, tpt, nbmax, nbs;
+  float scale_log2;
+  float* lse;
+  float* block_score;
+  float* block_lse;
+  float* ws;
+  int* status;
+  long long wait_ns;
+};
+
+struct Shared {
+  uint64_t kfull[kStages], kempty[kStages];
+  uint64_t qhi_full, qhi_empty, qlo_full, drain;
+  uint64_t sfull[2], sempty[2];
+  uint64_t epi;  // epilogue rendezvous of the 128 softmax threads
+  int prefix[kMaxDocs + 1];
+  float red[4][32];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+constexpr size_t kSmemBytes = 1024 + (size_t)(kStages + kMaxQhi) * kStageBytes + sizeof(Shared);
+
+struct Tile {
+  int t0, tend, bos;
+};
+
+__device__ __forceinline__ Tile tile_of(int g, const int* prefix, int nd, const int32_t* cu,
+                                        int tpt) {
+  int lo = 0, hi = nd;  // last d with prefix[d] <= g
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= g) lo = mid; else hi = mid;
+  }
+  const int local = g - prefix[lo];
+  const int ntd = prefix[lo + 1] - prefix[lo];
+  const int li = ntd - 1 - local;  // longest tile of the document first
+  Tile t;
+  t.bos = __ldg(cu + lo);
+  t.t0 = t.bos + li * tpt;
+  t.tend = min(t.t0 + tpt, (int)__ldg(cu + lo + 1));
+  return t;
+}
+
+__device__ __forceinline__ bool aborted(Shared* sh) {
+  return *reinterpret_cast<volatile int*>(&sh->abort_flag) != 0;
+}
+
+__device__ __forceinline__ void give_up(Shared* sh, int* status) {
+  record_status(status, HS_ERR_TIMEOUT);
+  *reinterpret_cast<volatile int*>(&sh->abort_flag) = 1;
+}
+
+// Sum of v[i] over the 32 lanes of the warp, delivered to lane i.
+__device__ __forceinline__ float transpose_reduce_sum(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < off; ++j) {
+      const float send = upper ? v[j] : v[j + off];
+      const float keep = upper ? v[j + off] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
+
+template <int B>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
+                      const __grid_constant__ CUtensorMap qmap, const BSParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* stages = base;
+  uint8_t* qhi = base + kStages * kStageBytes;
+  Shared* sh = reinterpret_cast<Shared*>(qhi + kMaxQhi * kStageBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nd = p.num_docs;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh->kfull[s], 1);
+      mbar_init(&sh->kempty[s], 1);
+    }
+    mbar_init(&sh->qhi_full, 1);
+    mbar_init(&sh->qhi_empty, 1);
+    mbar_init(&sh->qlo_full, 128);
+    mbar_init(&sh->drain, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh->sfull[b], 1);
+      mbar_init(&sh->sempty[b], 128);
+    }
+    mbar_init(&sh->epi, 128);
+    fence_barrier_init();
+    sh->abort_flag = 0;
+    // tiles per document (validating cu_seqlens on the way)
+    bool bad = __ldg(p.cu) != 0 || __ldg(p.cu + nd) != p.T;
+    int acc = 0;
+    sh->prefix[0] = 0;
+    for (int d = 0; d < nd; ++d) {
+      const int b0 = __ldg(p.cu + d), e0 = __ldg(p.cu + d + 1);
+      const int len = e0 - b0;
+      if (b0 < 0 || len < 0 || len > p.max_seqlen || e0 > p.T) bad = true;
+      else acc += (len + p.tpt - 1) / p.tpt;
+      sh->prefix[d + 1] = acc;
+    }
+    if (bad) record_status(p.status, HS_ERR_INVALID_ARG);
+  }
+  if (warp == 1) tmem_alloc(&sh->tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+  const int total = sh->prefix[nd];
+  const int G = gridDim.x, cta = blockIdx.x;
+  const long long lim = p.wait_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&qmap);
+      int fills[kStages];
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) fills[s] = 0;
+      int qfills = 0;
+      uint32_t kst = 0, kph = 0;
+      for (int it = 0; it * G < total && !aborted(sh); ++it) {
+        const int g = it * G + ((it & 1) ? (G - 1 - cta) : cta);
+        if (g >= total) continue;
+        const Tile tl = tile_of(g, sh->prefix, nd, p.cu, p.tpt);
+        // warm L2 with the next tile's q rows (the softmax warps read them)
+        {
+          const int it2 = it + 1, g2 = it2 * G + ((it2 & 1) ? (G - 1 - cta) : cta);
+          if (g2 < total) {
+            const Tile t2 = tile_of(g2, sh->prefix, nd, p.cu, p.tpt);
+            for (int ch = 0; ch < p.nck; ++ch) tma_prefetch_3d(&qmap, ch * 64, 0, t2.t0);
+          }
+        }
+        if (p.nq_smem > 0) {
+          if (qfills > 0 && !mbar_wait(&sh->qhi_empty, (qfills - 1) & 1, lim)) {
+            give_up(sh, p.status);
+            break;
+          }
+          mbar_expect_tx(&sh->qhi_full, p.nq_smem * kStageBytes);
+          for (int j = 0; j < p.nq_smem; ++j)
+            tma_load_3d(qhi + j * kStageBytes, &qmap, &sh->qhi_full, (p.nq_tmem + j) * 64, 0,
+                        tl.t0);
+          ++qfills;
+        }
+        const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
+        for (int kt = 0; kt < nkt && !aborted(sh); ++kt) {
+          for (int ch = 0; ch < p.nck; ++ch) {
+            if (!mbar_wait(&sh->kempty[kst], kph ^ 1, lim)) {
+              give_up(sh, p.status);
+              break;
+            }
+            mbar_expect_tx(&sh->kfull[kst], kStageBytes);
+            tma_load_2d(stages + kst * kStageBytes, &kmap, &sh->kfull[kst], ch * 64,
+                        tl.bos + kt * kKeyTile);
+            ++fills[kst];
+            if (++kst == kStages) {
+              kst = 0;
+              kph ^= 1;
+            }
+          }
+        }
+      }
+      // no copy may still be landing when the CTA exits
+      for (int s = 0; s < kStages; ++s)
+        if (fills[s] > 0) mbar_wait(&sh->kfull[s], (fills[s] - 1) & 1, kDefaultWaitNs);
+      if (qfills > 0) mbar_wait(&sh->qhi_full, (qfills - 1) & 1, kDefaultWaitNs);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+      uint64_t qhi_desc[kMaxQhi];
+#pragma unroll
+      for (int j = 0; j < kMaxQhi; ++j)
+        qhi_desc[j] = umma_desc_sw128(smem_u32(qhi + j * kStageBytes), 16, 1024);
+      const uint64_t stage_desc0 = umma_desc_sw128(smem_u32(stages), 16, 1024);
+      uint32_t kst = 0, kph = 0, sidx = 0;
+      int qtile = 0;
+      bool issued = false;
+      for (int it = 0; it * G < total && !aborted(sh); ++it) {
+        const int g = it * G + ((it & 1) ? (G - 1 - cta) : cta);
+        if (g >= total) continue;
+        const Tile tl = tile_of(g, sh->prefix, nd, p.cu, p.tpt);
+        const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
+        if (!mbar_wait(&sh->qlo_full, qtile & 1, lim) ||
+            (p.nq_smem > 0 && !mbar_wait(&sh->qhi_full, qtile & 1, lim))) {
+          give_up(sh, p.status);
+          break;
+        }
+        tc_fence_after();
+        bool ok = true;
+        for (int kt = 0; kt < nkt && ok; ++kt) {
+          const uint32_t buf = sidx & 1, use = sidx >> 1;
+          if (!mbar_wait(&sh->sempty[buf], (use & 1) ^ 1, lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + kSCol + buf * 128;
+          for (int ch = 0; ch < p.nck; ++ch) {
+            if (!mbar_wait(&sh->kfull[kst], kph, lim)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // stage descriptors advance by 16 KB = 1024 address units
+            const uint64_t bdesc = stage_desc0 + (uint64_t)(kst * (kStageBytes >> 4));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t accum = (ch | k) != 0;
+              if (ch < p.nq_tmem)
+                umma_ts(d, tmem + ch * 32 + k * 8, bdesc + 2 * k, idesc, accum);
+              else
+                umma_ss(d, qhi_desc[ch - p.nq_tmem] + 2 * k, bdesc + 2 * k, idesc, accum);
+            }
+            issued = true;
+            umma_commit(&sh->kempty[kst]);
+            if (++kst == kStages) {
+              kst = 0;
+              kph ^= 1;
+            }
+          }
+          if (!ok) break;
+          umma_commit(&sh->sfull[buf]);
+          ++sidx;
+        }
+        if (!ok) {
+          give_up(sh, p.status);
+          break;
+        }
+        if (p.nq_smem > 0) umma_commit(&sh->qhi_empty);
+        ++qtile;
+      }
+      if (issued) {  // every MMA done before TMEM is released
+        umma_commit(&sh->drain);
+        mbar_wait(&sh->drain, 0, kDefaultWaitNs);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int g4 = warp & 3;
+    const int r = 32 * g4 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * g4) << 16);
+    const int H = p.H;
+    const int hp = H / 32;  // warps per token
+    uint32_t sidx = 0, epi_ph = 0;
+    for (int it = 0; it * G < total && !aborted(sh); ++it) {
+      const int g = it * G + ((it & 1) ? (G - 1 - cta) : cta);
+      if (g >= total) continue;
+      const Tile tl = tile_of(g, sh->prefix, nd, p.cu, p.tpt);
+      const int tok = tl.t0 + r / H;
+      const int h = r % H;
+      const bool valid = tok < tl.tend;
+      const int tok_c = valid ? tok : tl.tend - 1;  // invalid rows mirror a valid token
+      // 1. this row of q (first nq_tmem chunks) into TMEM; the previous
+      //    tile's MMAs have all completed (its last S buffer was observed).
+      {
+        const __nv_bfloat16* src = p.q + (int64_t)tok_c * p.qrs + (int64_t)h * p.qhs;
+        for (int ch = 0; ch < p.nq_tmem; ++ch) {
+          uint32_t v[32];
+          const uint4* s4 = reinterpret_cast<const uint4*>(src + ch * 64);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint4 x = __ldg(s4 + i);
+            v[4 * i + 0] = x.x;
+            v[4 * i + 1] = x.y;
+            v[4 * i + 2] = x.z;
+            v[4 * i + 3] = x.w;
+          }
+          tmem_st32(lane_base + ch * 32, v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sh->qlo_full);
+      }
+      // 2. key tiles
+      const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int kt = 0; kt < nkt; ++kt) {
+        const uint32_t buf = sidx & 1, use = sidx >> 1;
+        if (!mbar_wait(&sh->sfull[buf], use & 1, lim)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float x[kKeyTile];
+#pragma unroll
+        for (int j = 0; j < kKeyTile / 32; ++j) {
+          uint32_t u[32];
+          tmem_ld32(lane_base + kSCol + buf * 128 + j * 32, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[j * 32 + i] = __uint_as_float(u[i]);
+        }
+        tc_fence_before();
+        mbar_arrive(&sh->sempty[buf]);
+        ++sidx;
+        const int key0 = tl.bos + kt * kKeyTile;
+        if (key0 + kKeyTile - 1 > tl.t0) {  // the causal edge crosses this tile
+#pragma unroll
+          for (int c = 0; c < kKeyTile; ++c)
+            x[c] = (key0 + c <= tok_c) ? x[c] * p.scale_log2 : -INFINITY;
+        } else {
+#pragma unroll
+          for (int c = 0; c < kKeyTile; ++c) x[c] *= p.scale_log2;
+        }
+        float* wsr = p.ws + (size_t)blockIdx.x * p.nbmax * 128 + r;
+        const int b0 = kt * (kKeyTile / B);
+#pragma unroll
+        for (int blk = 0; blk < kKeyTile / B; ++blk) {
+          float bm = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < B; ++c) bm = fmaxf(bm, x[blk * B + c]);
+          float blse = -INFINITY;
+          if (bm != -INFINITY) {
+            float bs = 0.f;
+#pragma unroll
+            for (int c = 0; c < B; ++c) bs += fast_exp2(x[blk * B + c] - bm);
+            blse = bm + fast_log2(bs);
+            const float mn = fmaxf(m, bm);
+            l = l * fast_exp2(m - mn) + bs * fast_exp2(bm - mn);
+            m = mn;
+          }
+          if (b0 + blk < p.nbmax) wsr[(size_t)(b0 + blk) * 128] = blse;
+        }
+      }
+      if (!ok) {
+        give_up(sh, p.status);
+        break;
+      }
+      // 3. epilogue: row LSE, head-summed block mass, optional per-head block LSE
+      const float lse2 = m + fast_log2(l);
+      if (valid) p.lse[(int64_t)tok * H + h] = lse2 * kLn2;
+      const int bq = valid ? (tok - tl.bos) / B : -1;
+      const float* wsr = p.ws + (size_t)blockIdx.x * p.nbmax * 128 + r;
+      float* blo = (valid && p.block_lse) ? p.block_lse + ((int64_t)tok * H + h) * p.nbs : nullptr;
+      const int tk = g4 / hp;
+      const bool first = (g4 % hp) == 0;
+      const int tok_w = tl.t0 + tk;
+      for (int bb0 = 0; bb0 < p.nbmax; bb0 += 32) {
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int b = bb0 + j;
+          float e = 0.f;
+          if (b <= bq) {
+            const float w = wsr[(size_t)b * 128];
+            e = fast_exp2(w - lse2);
+            if (blo) blo[b] = w * kLn2;
+          } else if (blo && b < p.nbmax) {
+            blo[b] = -INFINITY;
+          }
+          v[j] = e;
+        }
+        const float s = transpose_reduce_sum(v);
+        sh->red[g4][lane] = s;
+        // bounded rendezvous (an aborted warp must not strand the others)
+        mbar_arrive(&sh->epi);
+        if (!mbar_wait(&sh->epi, epi_ph, lim)) {
+          ok = false;
+          break;
+        }
+        epi_ph ^= 1;
+        if (first && tok_w < tl.tend && bb0 + lane < p.nbmax) {
+          float acc = 0.f;
+          for (int i = 0; i < hp; ++i) acc += sh->red[g4 + i][lane];
+          p.block_score[(int64_t)tok_w * p.nbs + bb0 + lane] = acc;
+        }
+        mbar_arrive(&sh->epi);
+        if (!mbar_wait(&sh->epi, epi_ph, lim)) {
+          ok = false;
+          break;
+        }
+        epi_ph ^= 1;
+      }
+      if (!ok) {
+        give_up(sh, p.status);
+        break;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+int grid_for(int total_tokens, int num_docs, int num_heads) {
+  const int tpt = 128 / num_heads;
+  const long long tiles = (long long)(total_tokens + tpt - 1) / tpt + num_docs;
+  return (int)(tiles < sm_count() ? tiles : sm_count());
+}
+
+}  // namespace
+
+bool tc_block_score_supported(int num_heads, int dk, int block_size, int nbmax) {
+  (void)nbmax;
+  return (num_heads == 32 || num_heads == 64 || num_heads == 128) && dk % 64 == 0 &&
+         dk >= 64 && dk <= 64 * (kMaxTmemQ + kMaxQhi) &&
+         (block_size == 16 || block_size == 32 || block_size == 64 || block_size == 128);
+}
+
+size_t tc_block_score_workspace(int total_tokens, int num_docs, int num_heads, int nbmax) {
+  return (size_t)grid_for(total_tokens, num_docs, num_heads) * nbmax * 128 * sizeof(float);
+}
+
+// Data-dependent conditions of the tensor-core path (alignment, doc count).
+bool tc_block_score_eligible(const ScoreArgs& a) {
+  const Problem& p = a.p;
+  return p.num_docs <= kMaxDocs && (reinterpret_cast<uintptr_t>(p.q) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(p.k) & 15) == 0 && p.q_row_stride % 8 == 0 &&
+         p.q_head_stride % 8 == 0 && p.k_row_stride % 8 == 0;
+}
+
+cudaError_t launch_tc_block_score(const ScoreArgs& a, long long wait_limit, cudaStream_t s) {
+  const Problem& p = a.p;
+  CUtensorMap kmap, qmap;
+  {
+    const uint64_t dims[2] = {(uint64_t)p.dk, (uint64_t)p.total_tokens};
+    const uint64_t strides[1] = {(uint64_t)p.k_row_stride * 2};
+    const uint32_t box[2] = {64, kKeyTile};
+    if (!encode_bf16_map(&kmap, p.k, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  const int tpt = 128 / p.num_heads;
+  {
+    const uint64_t dims[3] = {(uint64_t)p.dk, (uint64_t)p.num_heads, (uint64_t)p.total_tokens};
+    const uint64_t strides[2] = {(uint64_t)p.q_head_stride * 2, (uint64_t)p.q_row_stride * 2};
+    const uint32_t box[3] = {64, (uint32_t)p.num_heads, (uint32_t)tpt};
+    if (!encode_bf16_map(&qmap, p.q, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  BSParams bp;
+  bp.cu = p.cu_seqlens;
+  bp.num_docs = p.num_docs;
+  bp.T = p.total_tokens;
+  bp.max_seqlen = p.max_seqlen;
+  bp.q = static_cast<const __nv_bfloat16*>(p.q);
+  bp.qrs = p.q_row_stride;
+  bp.qhs = p.q_head_stride;
+  bp.H = p.num_heads;
+  bp.nck = p.dk / 64;
+  bp.nq_tmem = bp.nck < kMaxTmemQ ? bp.nck : kMaxTmemQ;
+  bp.nq_smem = bp.nck - bp.nq_tmem;
+  bp.tpt = tpt;
+  bp.nbmax = a.nbmax;
+  bp.nbs = a.nb_stride;
+  bp.scale_log2 = p.scale * kLog2e;
+  bp.lse = a.lse;
+  bp.block_score = a.block_score;
+  bp.block_lse = a.block_lse;
+  bp.ws = static_cast<float*>(a.workspace);
+  bp.status = p.status;
+  bp.wait_ns = wait_limit > 0 ? wait_limit : kDefaultWaitNs;
+  const int grid = grid_for(p.total_tokens, p.num_docs, p.num_heads);
+  void (*kern)(const CUtensorMap, const CUtensorMap, const BSParams) = nullptr;
+  switch (a.block_size) {
+    case 16: kern = tc_block_score_kernel<16>; break;
+    case 32: kern = tc_block_score_kernel<32>; break;
+    case 64: kern = tc_block_score_kernel<64>; break;
+    default: kern = tc_block_score_kernel<128>; break;
+  }
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, kSmemBytes, s>>>(kmap, qmap, bp);
+  return cudaGetLastError();
+}
+
+}  // namespace hs

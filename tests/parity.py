@@ -45,7 +45,8 @@ def check_lse(gpu, ref, what="lse", tol=LSE_ABS):
     r = np.asarray(ref, np.float64)
     assert g.shape == r.shape, (what, g.shape, r.shape)
     both_inf = np.isneginf(g) & np.isneginf(r)
-    err = np.where(both_inf, 0.0, np.abs(g - r))
+    with np.errstate(invalid="ignore"):
+        err = np.where(both_inf, 0.0, np.abs(g - r))
     mx = float(np.nanmax(err)) if err.size else 0.0
     assert not np.any(np.isnan(err)), what + ": NaN"
     assert mx <= tol, "%s max abs err %.3e > %.1e" % (what, mx, tol)
