@@ -174,17 +174,17 @@ simt_attention_kernel(AttnArgs a) {
     nseg = (t + 1 - wlo + 127) / 128;
   }
   const int bq = (t - bos) / a.block_size;
-  int prev = -1;
   for (int sgi = 0; sgi < nseg; ++sgi) {
     int lo, hi;
     if (kSparse) {
-      const int b = __ldg(a.idx + (int64_t)t * a.topk + sgi);
+      // a block id must lie in [0, bq] and exceed the entry before it
+      const int32_t* row = a.idx + (int64_t)t * a.topk;
+      const int b = __ldg(row + sgi);
       if (b < 0) continue;
-      if (b > bq || b <= prev) {
+      if (b > bq || (sgi > 0 && b <= __ldg(row + sgi - 1))) {
         if (tid == 0) record_status(p.status, HS_ERR_INVALID_INDEX);
         continue;
       }
-      prev = b;
       lo = bos + b * a.block_size;
       hi = min(lo + a.block_size, t + 1);
     } else {

@@ -27,8 +27,9 @@
 // rescales O^T in TMEM), write P^T as bf16 into one 128-byte-swizzled buffer
 // and accumulate per-head sums in registers.  The sink joins in the
 // epilogue, which reads O^T back per dv row and writes out[t, h, :].
-// Warp 0 = TMA producer, warp 1 = MMA issuer / TMEM owner, warps 2-5 =
-// softmax + epilogue.  All waits are bounded (HS_ERR_TIMEOUT, drain, free).
+// Warp 0 = TMA producer, warp 1 = MMA issuer / TMEM owner, warps 2-9 = two
+// softmax warpgroups, each owning 32 of the 64 heads (per-head state never
+// crosses warpgroups).  All waits are bounded (HS_ERR_TIMEOUT, drain, free).
 
 #include <math.h>
 
@@ -42,7 +43,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA, 2 softmax warpgroups
 constexpr int kH = 64;              // heads (N of every MMA)
 constexpr int kTile = 128;          // keys per tile (M of the QK MMA)
 constexpr int kSlots = 4;           // ring slots
@@ -74,12 +75,15 @@ struct Shared {
   uint64_t full[kSlots], empty[kSlots];
   uint64_t qfull[kMaxQChunks], qempty[kMaxQChunks];
   uint64_t sfull[2], sempty[2];
-  uint64_t pfull, pvdone, ofull, oempty, rv, drain;
-  float red[4][kH];
-  float mrun[kH];
-  float alpha[kH];
-  float lsum[kH];
-  int rescale[2];  // per tile parity: some head's running max rose
+  uint64_t pfull, pvdone, ofull, oempty, drain;
+  uint64_t rv[2];            // rendezvous inside softmax warpgroup wg (128 threads)
+  float red[2][4][32];       // [warpgroup][warp][lane] partial reductions
+  float mrun[kH];            // running max per head (log2 domain)
+  float alpha[kH];           // rescale factor per head
+  float lsum[kH];            // output multiplier per head
+  int rescale[2][2];         // [warpgroup][tile parity]: some head's max rose
+  int plist[256];            // producer's selected-block list of its token
+  int blist[2][256];         // each softmax warpgroup's list of its token
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -106,6 +110,15 @@ struct TokenPlan {
   int ntile;
 };
 
+// Index rule shared by every role: entry s of idx[t] is a selected block when
+// 0 <= b <= bq(t) and b is larger than the raw entry before it (ascending,
+// no duplicates; -1 padding fails the first test).  Rows that break it get
+// the offending entries skipped and HS_ERR_INVALID_INDEX reported.
+__device__ __forceinline__ bool entry_ok(const int32_t* row, int s, int bq, int& b) {
+  b = __ldg(row + s);
+  return b >= 0 && b <= bq && (s == 0 || b > __ldg(row + s - 1));
+}
+
 template <bool kSparse>
 __device__ __forceinline__ TokenPlan plan_token(const AttnParams& p, int t, bool report) {
   TokenPlan tp;
@@ -119,17 +132,12 @@ __device__ __forceinline__ TokenPlan plan_token(const AttnParams& p, int t, bool
   if (!tp.ok) return tp;
   if (kSparse) {
     const int32_t* row = p.idx + (int64_t)t * p.topk;
-    int prev = -1, n = 0;
+    int n = 0;
     bool bad = false;
     for (int s = 0; s < p.topk; ++s) {
-      const int b = __ldg(row + s);
-      if (b < 0) continue;
-      if (b > tp.bq || b <= prev) {
-        bad = true;
-        continue;
-      }
-      prev = b;
-      ++n;
+      int b;
+      if (entry_ok(row, s, tp.bq, b)) ++n;
+      else if (b >= 0) bad = true;
     }
     if (bad && report) record_status(p.status, HS_ERR_INVALID_INDEX);
     tp.nsel = n;
@@ -141,21 +149,6 @@ __device__ __forceinline__ TokenPlan plan_token(const AttnParams& p, int t, bool
     tp.ntile = (tp.nkeys + kTile - 1) / kTile;
   }
   return tp;
-}
-
-// The n-th valid selected block of token t (same validation as plan_token),
-// or the own block when n is past the last one (a masked filler slot).
-__device__ __forceinline__ int nth_block(const AttnParams& p, int t, int bq, int n) {
-  const int32_t* row = p.idx + (int64_t)t * p.topk;
-  int prev = -1, k = 0;
-  for (int s = 0; s < p.topk; ++s) {
-    const int b = __ldg(row + s);
-    if (b < 0 || b > bq || b <= prev) continue;
-    prev = b;
-    if (k == n) return b;
-    ++k;
-  }
-  return bq;
 }
 
 // 32-lane transpose reductions: lane i receives op over lanes of v[i].
@@ -188,10 +181,10 @@ __device__ __forceinline__ float tr_sum(float (&v)[32]) {
   return v[0];
 }
 
-// Bounded rendezvous of the 128 softmax threads.
-__device__ __forceinline__ bool rendezvous(Shared* sh, uint32_t& ph, long long lim) {
-  mbar_arrive(&sh->rv);
-  const bool ok = mbar_wait(&sh->rv, ph, lim);
+// Bounded rendezvous of the 128 threads of softmax warpgroup wg.
+__device__ __forceinline__ bool rendezvous(Shared* sh, int wg, uint32_t& ph, long long lim) {
+  mbar_arrive(&sh->rv[wg]);
+  const bool ok = mbar_wait(&sh->rv[wg], ph, lim);
   ph ^= 1;
   return ok;
 }
@@ -221,17 +214,17 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->sfull[b], 1);
-      mbar_init(&sh->sempty[b], 128);
+      mbar_init(&sh->sempty[b], 256);
+      mbar_init(&sh->rv[b], 128);
     }
-    mbar_init(&sh->pfull, 128);
+    mbar_init(&sh->pfull, 256);
     mbar_init(&sh->pvdone, 1);
     mbar_init(&sh->ofull, 1);
-    mbar_init(&sh->oempty, 128);
-    mbar_init(&sh->rv, 128);
+    mbar_init(&sh->oempty, 256);
     mbar_init(&sh->drain, 1);
     fence_barrier_init();
     sh->abort_flag = 0;
-    sh->rescale[0] = sh->rescale[1] = 0;
+    sh->rescale[0][0] = sh->rescale[0][1] = sh->rescale[1][0] = sh->rescale[1][1] = 0;
   }
   if (warp == 1) tmem_alloc(&sh->tmem_base, 512);
   tc_fence_before();
@@ -265,7 +258,8 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           for (int j = 0; j < per; ++j) {
             int row0;
             if (kSparse) {
-              const int b = nth_block(p, t, tp.bq, tile * per + j);
+              const int slotn = tile * per + j;  // past the list: masked filler (own block)
+              const int b = slotn < tp.nsel ? sh->plist[slotn] : tp.bq;
               row0 = tp.bos + b * p.B;
             } else {
               row0 = tp.wlo + tile * kTile;
@@ -285,6 +279,14 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       for (int t = blockIdx.x; t < p.T && !stop; t += G) {
         const TokenPlan tp = plan_token<kSparse>(p, t, true);
         if (!tp.ok || tp.ntile == 0) continue;
+        if (kSparse) {  // this token's selected blocks, once
+          const int32_t* row = p.idx + (int64_t)t * p.topk;
+          int n = 0;
+          for (int s2 = 0; s2 < p.topk; ++s2) {
+            int b;
+            if (entry_ok(row, s2, tp.bq, b)) sh->plist[n++] = b;
+          }
+        }
         // Q_t chunks, each as soon as the previous token's last QK released it
         for (int c = 0; c < p.nck; ++c) {
           if (qfills[c] > 0 && !mbar_wait(&sh->qempty[c], (qfills[c] - 1) & 1, lim)) {
@@ -400,37 +402,52 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    // Two warpgroups; warpgroup wg owns heads [32 wg, 32 wg + 32).  Thread
+    // (warp, lane) owns key row r of S^T and value row r of each O^T chunk.
+    const int wg = (warp - 2) >> 2;
     const int g4 = warp & 3;
-    const int r = 32 * g4 + lane;  // key row of S^T / dv row of O^T
+    const int r = 32 * g4 + lane;
+    const int hb = 32 * wg;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * g4) << 16);
+    const float sl2 = p.scale_log2;
+    const int dvs = p.nvc * 128;
     uint32_t sidx = 0, npv = 0, rvph = 0, ntok = 0, gt = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.T && ok && !aborted(sh); t += G) {
       const TokenPlan tp = plan_token<kSparse>(p, t, false);
       if (!tp.ok) continue;
       if (tp.ntile == 0) {  // no valid block: empty softmax, only the sink
-        const int dvs = p.nvc * 128;
-        for (int e = r; e < kH * dvs; e += 128)
-          p.out[(int64_t)t * kH * dvs + e] = __float2bfloat16_rn(0.f);
-        if (r < kH) p.lse[(int64_t)t * kH + r] = p.sink ? __ldg(p.sink + r) : -INFINITY;
+        for (int e = r; e < 32 * dvs; e += 128)
+          p.out[((int64_t)t * kH + hb) * dvs + e] = __float2bfloat16_rn(0.f);
+        if (r < 32) p.lse[(int64_t)t * kH + hb + r] = p.sink ? __ldg(p.sink + hb + r) : -INFINITY;
         continue;
       }
-      float lpart[kH];
+      if (kSparse) {  // compact this token's selected blocks (warp 0 of the group)
+        if (g4 == 0) {
+          const int32_t* row = p.idx + (int64_t)t * p.topk;
+          int n = 0;
+          for (int base0 = 0; base0 < p.topk; base0 += 32) {
+            const int s2 = base0 + lane;
+            int b = -1;
+            const bool v = s2 < p.topk && entry_ok(row, s2, tp.bq, b);
+            const unsigned mask = __ballot_sync(0xffffffffu, v);
+            if (v) sh->blist[wg][n + __popc(mask & ((1u << lane) - 1u))] = b;
+            n += __popc(mask);
+          }
+        }
+        if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
+      }
+      float lpart[32];
 #pragma unroll
-      for (int h = 0; h < kH; ++h) lpart[h] = 0.f;
+      for (int k = 0; k < 32; ++k) lpart[k] = 0.f;
       for (int i = 0; i < tp.ntile && ok; ++i) {
         const uint32_t buf = sidx & 1, use = sidx >> 1;
         if (!mbar_wait(&sh->sfull[buf], use & 1, lim)) { ok = false; break; }
         tc_fence_after();
-        float x[kH];
-#pragma unroll
-        for (int j = 0; j < kH / 32; ++j) {
-          uint32_t u[32];
-          tmem_ld32(lane_base + kSCol + buf * kH + j * 32, u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) x[j * 32 + k] = __uint_as_float(u[k]);
-        }
+        uint32_t u[32];
+        tmem_ld32(lane_base + kSCol + buf * kH + hb, u);
+        tmem_ld_wait();
+        reg_fence(u);
         tc_fence_before();
         mbar_arrive(&sh->sempty[buf]);
         ++sidx;
@@ -438,89 +455,80 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         bool valid;
         if (kSparse) {
           const int slotn = i * (kTile / p.B) + r / p.B;
-          const int b = nth_block(p, t, tp.bq, slotn);
+          const int b = slotn < tp.nsel ? sh->blist[wg][slotn] : tp.bq;
           const int key = tp.bos + b * p.B + (r % p.B);
           valid = slotn < tp.nsel && key <= t;
         } else {
-          const int key = tp.wlo + i * kTile + r;
-          valid = key <= t;
+          valid = tp.wlo + i * kTile + r <= t;
         }
+        float x[32];
 #pragma unroll
-        for (int h = 0; h < kH; ++h) x[h] = valid ? x[h] * p.scale_log2 : -INFINITY;
-        // per-head max over the 128 rows
+        for (int k = 0; k < 32; ++k) x[k] = valid ? __uint_as_float(u[k]) * sl2 : -INFINITY;
+        // per-head max over the 128 key rows
         {
-          float a[32], b2[32];
+          float a[32];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            a[k] = x[k];
-            b2[k] = x[k + 32];
-          }
-          const float m0 = tr_max(a), m1 = tr_max(b2);
-          sh->red[g4][lane] = m0;
-          sh->red[g4][lane + 32] = m1;
+          for (int k = 0; k < 32; ++k) a[k] = x[k];
+          sh->red[wg][g4][lane] = tr_max(a);
         }
-        if (!rendezvous(sh, rvph, lim)) { ok = false; break; }
-        if (r < kH) {
-          const float tm = fmaxf(fmaxf(sh->red[0][r], sh->red[1][r]),
-                                 fmaxf(sh->red[2][r], sh->red[3][r]));
-          float mo = (i == 0) ? -INFINITY : sh->mrun[r];
+        if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
+        if (g4 == 0) {
+          const int hh = hb + lane;
+          const float tm = fmaxf(fmaxf(sh->red[wg][0][lane], sh->red[wg][1][lane]),
+                                 fmaxf(sh->red[wg][2][lane], sh->red[wg][3][lane]));
+          const float mo = (i == 0) ? -INFINITY : sh->mrun[hh];
           float mn = mo;
-          if (i == 0) mn = tm;
-          else if (tm > mo + kRescaleLog2) mn = tm;
-          // a head whose keys are all masked so far keeps -inf: use 0 as
-          // reference so that exp2 stays finite (all its P are zero anyway)
-          sh->alpha[r] = (i == 0 || mn == mo) ? 1.f : fast_exp2(mo - mn);
-          sh->mrun[r] = mn;
-          if (i > 0 && mn != mo) sh->rescale[gt & 1] = 1;
+          if (i == 0 || tm > mo + kRescaleLog2) mn = tm;
+          sh->alpha[hh] = (i == 0 || mn == mo) ? 1.f : fast_exp2(mo - mn);
+          sh->mrun[hh] = mn;
+          if (i > 0 && mn != mo) sh->rescale[wg][gt & 1] = 1;
+          // the other parity's flag was last read before this rendezvous
+          if (lane == 0) sh->rescale[wg][(gt + 1) & 1] = 0;
         }
-        // the other parity's flag was last read before the rendezvous above
-        if (r == 0) sh->rescale[(gt + 1) & 1] = 0;
-        if (!rendezvous(sh, rvph, lim)) { ok = false; break; }
-        const bool resc = i > 0 && sh->rescale[gt & 1] != 0;
+        if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
+        const bool resc = i > 0 && sh->rescale[wg][gt & 1] != 0;
         ++gt;
-        // P^T may be written once PV of the previous tile has read it
+        // P^T may be rewritten once PV of the previous tile has read it
         if (i > 0) {
           if (!mbar_wait(&sh->pvdone, npv & 1, lim)) { ok = false; break; }
           ++npv;
           tc_fence_after();
         }
-        if (resc) {
-          // rare: the running max of some head rose; rescale O^T columns
+        if (resc) {  // rare: some head's running max rose; rescale its O^T columns
 #pragma unroll 1
           for (int c = 0; c < p.nvc; ++c) {
+            uint32_t w[32];
+            const uint32_t ta = lane_base + c * kH + hb;
+            tmem_ld32(ta, w);
+            tmem_ld_wait();
+            reg_fence(w);
 #pragma unroll
-            for (int j = 0; j < kH / 32; ++j) {
-              uint32_t u[32];
-              const uint32_t ta = lane_base + c * kH + j * 32;
-              tmem_ld32(ta, u);
-              tmem_ld_wait();
-#pragma unroll
-              for (int k = 0; k < 32; ++k)
-                u[k] = __float_as_uint(__uint_as_float(u[k]) * sh->alpha[j * 32 + k]);
-              tmem_st32(ta, u);
-            }
+            for (int k = 0; k < 32; ++k)
+              w[k] = __float_as_uint(__uint_as_float(w[k]) * sh->alpha[hb + k]);
+            tmem_st32(ta, w);
           }
           tmem_st_wait();
 #pragma unroll
-          for (int h = 0; h < kH; ++h) lpart[h] *= sh->alpha[h];
+          for (int k = 0; k < 32; ++k) lpart[k] *= sh->alpha[hb + k];
         }
-        // P^T row r: exp2(x - m_h) as bf16, 128-byte swizzled (MN-major B)
+        // P^T row r, heads hb..hb+31: exp2(x - m_h) as bf16, 128-byte swizzled
         uint8_t* prow = pbuf + r * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t w[4];
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t w4[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int h0 = c * 8 + 2 * k;
-            const float mh0 = sh->mrun[h0], mh1 = sh->mrun[h0 + 1];
-            const float e0 = fast_exp2(x[h0] - (mh0 == -INFINITY ? 0.f : mh0));
-            const float e1 = fast_exp2(x[h0 + 1] - (mh1 == -INFINITY ? 0.f : mh1));
+            const int h0 = q4 * 8 + 2 * k;
+            const float e0 = fast_exp2(x[h0] - sh->mrun[hb + h0]);
+            const float e1 = fast_exp2(x[h0 + 1] - sh->mrun[hb + h0 + 1]);
             lpart[h0] += e0;
             lpart[h0 + 1] += e1;
             __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
-            w[k] = *reinterpret_cast<uint32_t*>(&pr);
+            w4[k] = *reinterpret_cast<uint32_t*>(&pr);
           }
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          const int cidx = 4 * wg + q4;
+          *reinterpret_cast<uint4*>(prow + ((cidx ^ (r & 7)) << 4)) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
@@ -528,55 +536,41 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       }
       if (!ok) break;
       // ---------------- epilogue: per-head sums, sink, normalisation
-      {
-        float a[32], b2[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          a[k] = lpart[k];
-          b2[k] = lpart[k + 32];
-        }
-        const float s0 = tr_sum(a), s1 = tr_sum(b2);
-        sh->red[g4][lane] = s0;
-        sh->red[g4][lane + 32] = s1;
-      }
-      if (!rendezvous(sh, rvph, lim)) { ok = false; break; }
-      if (r < kH) {
-        const float l = (sh->red[0][r] + sh->red[1][r]) + (sh->red[2][r] + sh->red[3][r]);
-        const float mh = sh->mrun[r];
-        const float m = (mh == -INFINITY) ? 0.f : mh;  // log2 reference used for P
-        const float sk = p.sink ? __ldg(p.sink + r) * kLog2e : -INFINITY;
+      sh->red[wg][g4][lane] = tr_sum(lpart);
+      if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
+      if (g4 == 0) {
+        const int hh = hb + lane;
+        const float l = (sh->red[wg][0][lane] + sh->red[wg][1][lane]) +
+                        (sh->red[wg][2][lane] + sh->red[wg][3][lane]);
+        const float m = sh->mrun[hh];  // finite: tile 0 always holds a valid key
+        const float sk = p.sink ? __ldg(p.sink + hh) * kLog2e : -INFINITY;
         const float M = fmaxf(m, sk);
         const float den = l * fast_exp2(m - M) + fast_exp2(sk - M);
-        sh->lsum[r] = fast_exp2(m - M) / den;  // multiplier of O
-        p.lse[(int64_t)t * kH + r] = (M + fast_log2(den)) * kLn2;
+        sh->lsum[hh] = fast_exp2(m - M) / den;
+        p.lse[(int64_t)t * kH + hh] = (M + fast_log2(den)) * kLn2;
       }
       // the last PV of this token must be complete before O^T is read
       if (!mbar_wait(&sh->pvdone, npv & 1, lim)) { ok = false; break; }
       ++npv;
       if (!mbar_wait(&sh->ofull, ntok & 1, lim)) { ok = false; break; }
       tc_fence_after();
-      if (!rendezvous(sh, rvph, lim)) { ok = false; break; }
-      __nv_bfloat16* orow = p.out + (int64_t)t * kH * (p.nvc * 128);
-      const int dvs = p.nvc * 128;
+      if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
+      __nv_bfloat16* orow = p.out + ((int64_t)t * kH + hb) * dvs;
       for (int c = 0; c < p.nvc; ++c) {
+        uint32_t w[32];
+        tmem_ld32(lane_base + c * kH + hb, w);
+        tmem_ld_wait();
+        reg_fence(w);
 #pragma unroll
-        for (int j = 0; j < kH / 32; ++j) {
-          uint32_t u[32];
-          tmem_ld32(lane_base + c * kH + j * 32, u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int h = j * 32 + k;
-            orow[(int64_t)h * dvs + c * 128 + r] =
-                __float2bfloat16_rn(__uint_as_float(u[k]) * sh->lsum[h]);
-          }
-        }
+        for (int k = 0; k < 32; ++k)
+          orow[(int64_t)k * dvs + c * 128 + r] =
+              __float2bfloat16_rn(__uint_as_float(w[k]) * sh->lsum[hb + k]);
       }
       tc_fence_before();
       mbar_arrive(&sh->oempty);
       ++ntok;
-      // lsum / mrun are rewritten for the next token only after everyone is done
-      if (!rendezvous(sh, rvph, lim)) { ok = false; break; }
+      // lsum / mrun / blist are rewritten for the next token only after this
+      if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
     }
     if (!ok) give_up(sh, p.status);
   }

@@ -25,9 +25,13 @@
 //    L2 resident).  At the end of the tile each row has its LSE; the head
 //    sum of exp2(blockLSE - LSE) is a 32-lane transpose-reduction per warp
 //    plus a fixed-order sum over the warps of a token (deterministic).
-//  * Warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner), warps 2-5
-//    = softmax / Q loader / epilogue.  Every wait is bounded; a timeout
-//    records HS_ERR_TIMEOUT, drains in-flight copies and MMAs, frees TMEM.
+//  * Warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner), warps 2-9
+//    = two softmax warpgroups that take alternate S tiles (one S buffer
+//    each), load q into TMEM and share the epilogue.  Per-row running
+//    (max, sum) pairs of the two warpgroups are merged at the end of the
+//    tile; S is read in 32-column chunks with the next tcgen05.ld in flight.
+//    Every wait is bounded; a timeout records HS_ERR_TIMEOUT, drains
+//    in-flight copies and MMAs, frees TMEM.
 
 #include <math.h>
 
@@ -41,7 +45,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA, 2 softmax warpgroups
 constexpr int kStages = 8;
 constexpr int kKeyTile = 128;
 constexpr int kStageBytes = kKeyTile * 64 * 2;  // 128 keys x 64 bf16
@@ -71,9 +75,11 @@ struct Shared {
   uint64_t kfull[kStages], kempty[kStages];
   uint64_t qhi_full, qhi_empty, qlo_full, drain;
   uint64_t sfull[2], sempty[2];
-  uint64_t epi;  // epilogue rendezvous of the 128 softmax threads
+  uint64_t epi_all;    // rendezvous of both softmax warpgroups (256 threads)
+  uint64_t epi_wg[2];  // rendezvous inside one warpgroup (128 threads)
   int prefix[kMaxDocs + 1];
-  float red[4][32];
+  float ml[2][2][2][128];  // [tile parity][warpgroup][max | sum][row]
+  float red[2][4][32];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -146,13 +152,15 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
     }
     mbar_init(&sh->qhi_full, 1);
     mbar_init(&sh->qhi_empty, 1);
-    mbar_init(&sh->qlo_full, 128);
+    mbar_init(&sh->qlo_full, 256);
     mbar_init(&sh->drain, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->sfull[b], 1);
       mbar_init(&sh->sempty[b], 128);
     }
-    mbar_init(&sh->epi, 128);
+    mbar_init(&sh->epi_all, 256);
+    mbar_init(&sh->epi_wg[0], 128);
+    mbar_init(&sh->epi_wg[1], 128);
     fence_barrier_init();
     sh->abort_flag = 0;
     // tiles per document (validating cu_seqlens on the way)
@@ -306,114 +314,184 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
     }
   } else {
     // ------------------------------------------------------------ softmax
+    // Two warpgroups; warpgroup wg owns S buffer wg, i.e. every other S tile.
+    // Per-row (max, sum) pairs are combined at the end of the query tile.
+    const int wg = (warp - 2) >> 2;
     const int g4 = warp & 3;
     const int r = 32 * g4 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * g4) << 16);
     const int H = p.H;
     const int hp = H / 32;  // warps per token
-    uint32_t sidx = 0, epi_ph = 0;
-    for (int it = 0; it * G < total && !aborted(sh); ++it) {
-      const int g = it * G + ((it & 1) ? (G - 1 - cta) : cta);
-      if (g >= total) continue;
-      const Tile tl = tile_of(g, sh->prefix, nd, p.cu, p.tpt);
+    const float sl2 = p.scale_log2;
+    float* const ws_row = p.ws + (size_t)blockIdx.x * p.nbmax * 128 + r;
+    uint32_t sbase = 0, all_ph = 0, wg_ph = 0;
+    bool ok = true;
+    // q rows of a tile into TMEM (this warpgroup's half of the chunks)
+    auto load_qlo = [&](const Tile& tq) {
+      const int tk = min(tq.t0 + r / H, tq.tend - 1);
+      const __nv_bfloat16* src = p.q + (int64_t)tk * p.qrs + (int64_t)(r % H) * p.qhs;
+      const int half = (p.nq_tmem + 1) >> 1;
+      const int c0 = wg ? half : 0, c1 = wg ? p.nq_tmem : half;
+      for (int ch = c0; ch < c1; ++ch) {
+        uint32_t v[32];
+        const uint4* s4 = reinterpret_cast<const uint4*>(src + ch * 64);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 x = __ldg(s4 + i);
+          v[4 * i + 0] = x.x;
+          v[4 * i + 1] = x.y;
+          v[4 * i + 2] = x.z;
+          v[4 * i + 3] = x.w;
+        }
+        tmem_st32(lane_base + ch * 32, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&sh->qlo_full);
+    };
+    auto tile_at = [&](int it2, Tile& out) -> bool {
+      if (it2 * G >= total) return false;
+      const int g2 = it2 * G + ((it2 & 1) ? (G - 1 - cta) : cta);
+      if (g2 >= total) return false;
+      out = tile_of(g2, sh->prefix, nd, p.cu, p.tpt);
+      return true;
+    };
+    Tile cur;
+    bool have = tile_at(0, cur);
+    if (have) load_qlo(cur);
+    for (int it = 0; have && ok && !aborted(sh); ++it) {
+      const Tile tl = cur;
       const int tok = tl.t0 + r / H;
       const int h = r % H;
       const bool valid = tok < tl.tend;
-      const int tok_c = valid ? tok : tl.tend - 1;  // invalid rows mirror a valid token
-      // 1. this row of q (first nq_tmem chunks) into TMEM; the previous
-      //    tile's MMAs have all completed (its last S buffer was observed).
-      {
-        const __nv_bfloat16* src = p.q + (int64_t)tok_c * p.qrs + (int64_t)h * p.qhs;
-        for (int ch = 0; ch < p.nq_tmem; ++ch) {
-          uint32_t v[32];
-          const uint4* s4 = reinterpret_cast<const uint4*>(src + ch * 64);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint4 x = __ldg(s4 + i);
-            v[4 * i + 0] = x.x;
-            v[4 * i + 1] = x.y;
-            v[4 * i + 2] = x.z;
-            v[4 * i + 3] = x.w;
-          }
-          tmem_st32(lane_base + ch * 32, v);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&sh->qlo_full);
-      }
-      // 2. key tiles
+      const int tok_c = valid ? tok : tl.tend - 1;
       const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
-      float m = -INFINITY, l = 0.f;
-      bool ok = true;
+      float m = -INFINITY, l = 0.f;  // log2 domain
       for (int kt = 0; kt < nkt; ++kt) {
-        const uint32_t buf = sidx & 1, use = sidx >> 1;
-        if (!mbar_wait(&sh->sfull[buf], use & 1, lim)) {
+        const uint32_t gs = sbase + kt;
+        if ((int)(gs & 1) != wg) continue;
+        if (!mbar_wait(&sh->sfull[wg], (gs >> 1) & 1, lim)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        float x[kKeyTile];
-#pragma unroll
-        for (int j = 0; j < kKeyTile / 32; ++j) {
-          uint32_t u[32];
-          tmem_ld32(lane_base + kSCol + buf * 128 + j * 32, u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[j * 32 + i] = __uint_as_float(u[i]);
-        }
-        tc_fence_before();
-        mbar_arrive(&sh->sempty[buf]);
-        ++sidx;
         const int key0 = tl.bos + kt * kKeyTile;
-        if (key0 + kKeyTile - 1 > tl.t0) {  // the causal edge crosses this tile
-#pragma unroll
-          for (int c = 0; c < kKeyTile; ++c)
-            x[c] = (key0 + c <= tok_c) ? x[c] * p.scale_log2 : -INFINITY;
-        } else {
-#pragma unroll
-          for (int c = 0; c < kKeyTile; ++c) x[c] *= p.scale_log2;
-        }
-        float* wsr = p.ws + (size_t)blockIdx.x * p.nbmax * 128 + r;
-        const int b0 = kt * (kKeyTile / B);
-#pragma unroll
-        for (int blk = 0; blk < kKeyTile / B; ++blk) {
-          float bm = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < B; ++c) bm = fmaxf(bm, x[blk * B + c]);
+        const bool need_mask = key0 + kKeyTile - 1 > tl.t0;
+        const uint32_t sa = lane_base + kSCol + wg * 128;
+        float bm = -INFINITY, bs = 0.f;  // running block max (raw logits) and sum
+        auto finish_block = [&](int bidx) {
           float blse = -INFINITY;
           if (bm != -INFINITY) {
-            float bs = 0.f;
-#pragma unroll
-            for (int c = 0; c < B; ++c) bs += fast_exp2(x[blk * B + c] - bm);
-            blse = bm + fast_log2(bs);
-            const float mn = fmaxf(m, bm);
-            l = l * fast_exp2(m - mn) + bs * fast_exp2(bm - mn);
+            blse = fmaf(bm, sl2, fast_log2(bs));
+            const float mn = fmaxf(m, blse);
+            l = l * fast_exp2(m - mn) + fast_exp2(blse - mn);
             m = mn;
           }
-          if (b0 + blk < p.nbmax) wsr[(size_t)(b0 + blk) * 128] = blse;
-        }
+          const int bg = kt * (kKeyTile / B) + bidx;
+          if (bg < p.nbmax) ws_row[(size_t)bg * 128] = blse;
+          bm = -INFINITY;
+          bs = 0.f;
+        };
+        // one 32-column chunk of S (raw logits in u)
+        auto chunk = [&](int j, uint32_t (&u)[32]) {
+          if (need_mask) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (key0 + 32 * j + i > tok_c) u[i] = 0xff800000u;  // -inf
+          }
+          float (&x)[32] = reinterpret_cast<float (&)[32]>(u);
+          if (B >= 32) {
+            float cm = x[0];
+#pragma unroll
+            for (int i = 1; i < 32; ++i) cm = fmaxf(cm, x[i]);
+            if (cm > bm) {
+              bs *= fast_exp2((bm - cm) * sl2);
+              bm = cm;
+            }
+            if (bm != -INFINITY) {
+              const float nb = -bm * sl2;
+              float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+              for (int i = 0; i < 32; i += 2) {
+                a0 += fast_exp2(fmaf(x[i], sl2, nb));
+                a1 += fast_exp2(fmaf(x[i + 1], sl2, nb));
+              }
+              bs += a0 + a1;
+            }
+            if (((32 * j + 32) % B) == 0) finish_block((32 * j) / B);
+          } else {
+#pragma unroll
+            for (int hb = 0; hb < 32 / B; ++hb) {
+              float cm = x[hb * B];
+#pragma unroll
+              for (int i = 1; i < B; ++i) cm = fmaxf(cm, x[hb * B + i]);
+              bm = cm;
+              if (bm != -INFINITY) {
+                const float nb = -bm * sl2;
+                float a0 = 0.f;
+#pragma unroll
+                for (int i = 0; i < B; ++i) a0 += fast_exp2(fmaf(x[hb * B + i], sl2, nb));
+                bs = a0;
+              }
+              finish_block((32 * j) / B + hb);
+            }
+          }
+        };
+        uint32_t ua[32], ub[32];
+        tmem_ld32(sa, ua);
+        tmem_ld_wait();
+        reg_fence(ua);
+        tmem_ld32(sa + 32, ub);
+        chunk(0, ua);
+        tmem_ld_wait();
+        reg_fence(ub);
+        tmem_ld32(sa + 64, ua);
+        chunk(1, ub);
+        tmem_ld_wait();
+        reg_fence(ua);
+        tmem_ld32(sa + 96, ub);
+        chunk(2, ua);
+        tmem_ld_wait();
+        reg_fence(ub);
+        tc_fence_before();
+        mbar_arrive(&sh->sempty[wg]);  // whole tile is in registers
+        chunk(3, ub);
       }
-      if (!ok) {
-        give_up(sh, p.status);
-        break;
-      }
-      // 3. epilogue: row LSE, head-summed block mass, optional per-head block LSE
-      const float lse2 = m + fast_log2(l);
-      if (valid) p.lse[(int64_t)tok * H + h] = lse2 * kLn2;
+      if (!ok) break;
+      sbase += nkt;
+      // ---- combine the two warpgroups' row statistics
+      const int mb = it & 1;
+      sh->ml[mb][wg][0][r] = m;
+      sh->ml[mb][wg][1][r] = l;
+      mbar_arrive(&sh->epi_all);
+      if (!mbar_wait(&sh->epi_all, all_ph, lim)) { ok = false; break; }
+      all_ph ^= 1;
+      const float m0 = sh->ml[mb][0][0][r], l0 = sh->ml[mb][0][1][r];
+      const float m1 = sh->ml[mb][1][0][r], l1 = sh->ml[mb][1][1][r];
+      const float M = fmaxf(m0, m1);
+      const float L = (m0 == -INFINITY ? 0.f : l0 * fast_exp2(m0 - M)) +
+                      (m1 == -INFINITY ? 0.f : l1 * fast_exp2(m1 - M));
+      const float lse2 = M + fast_log2(L);
+      if (wg == 0 && valid) p.lse[(int64_t)tok * H + h] = lse2 * kLn2;
+      // every MMA of this tile is complete: the next tile's q may enter TMEM
+      have = tile_at(it + 1, cur);
+      if (have) load_qlo(cur);
+      // ---- head-summed block masses (and optional per-head block LSE)
       const int bq = valid ? (tok - tl.bos) / B : -1;
-      const float* wsr = p.ws + (size_t)blockIdx.x * p.nbmax * 128 + r;
       float* blo = (valid && p.block_lse) ? p.block_lse + ((int64_t)tok * H + h) * p.nbs : nullptr;
-      const int tk = g4 / hp;
+      const int tkw = g4 / hp;
       const bool first = (g4 % hp) == 0;
-      const int tok_w = tl.t0 + tk;
-      for (int bb0 = 0; bb0 < p.nbmax; bb0 += 32) {
+      const int tok_w = tl.t0 + tkw;
+      const int nbatch = (p.nbmax + 31) / 32;
+      for (int bi = wg; bi < nbatch; bi += 2) {
+        const int bb0 = bi * 32;
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int b = bb0 + j;
           float e = 0.f;
           if (b <= bq) {
-            const float w = wsr[(size_t)b * 128];
+            const float w = ws_row[(size_t)b * 128];
             e = fast_exp2(w - lse2);
             if (blo) blo[b] = w * kLn2;
           } else if (blo && b < p.nbmax) {
@@ -422,31 +500,21 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
           v[j] = e;
         }
         const float s = transpose_reduce_sum(v);
-        sh->red[g4][lane] = s;
-        // bounded rendezvous (an aborted warp must not strand the others)
-        mbar_arrive(&sh->epi);
-        if (!mbar_wait(&sh->epi, epi_ph, lim)) {
-          ok = false;
-          break;
-        }
-        epi_ph ^= 1;
+        sh->red[wg][g4][lane] = s;
+        mbar_arrive(&sh->epi_wg[wg]);
+        if (!mbar_wait(&sh->epi_wg[wg], wg_ph, lim)) { ok = false; break; }
+        wg_ph ^= 1;
         if (first && tok_w < tl.tend && bb0 + lane < p.nbmax) {
           float acc = 0.f;
-          for (int i = 0; i < hp; ++i) acc += sh->red[g4 + i][lane];
+          for (int i = 0; i < hp; ++i) acc += sh->red[wg][g4 + i][lane];
           p.block_score[(int64_t)tok_w * p.nbs + bb0 + lane] = acc;
         }
-        mbar_arrive(&sh->epi);
-        if (!mbar_wait(&sh->epi, epi_ph, lim)) {
-          ok = false;
-          break;
-        }
-        epi_ph ^= 1;
-      }
-      if (!ok) {
-        give_up(sh, p.status);
-        break;
+        mbar_arrive(&sh->epi_wg[wg]);
+        if (!mbar_wait(&sh->epi_wg[wg], wg_ph, lim)) { ok = false; break; }
+        wg_ph ^= 1;
       }
     }
+    if (!ok) give_up(sh, p.status);
   }
 
   tc_fence_before();

@@ -151,6 +151,14 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Pins the use of registers filled by an asynchronous tcgen05.ld after the
+// tcgen05.wait::ld that completes it (the compiler sees no dependency
+// between the two asm statements otherwise).
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 // 32 consecutive 32-bit TMEM columns written from this thread's registers.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(

@@ -165,8 +165,10 @@ hs_status hs_select_topk(const float* block_score, int nb_stride,
  * sink is in the scaled logit space (not multiplied by softmax_scale).
  *
  *   idx    [T, topk] int32: ascending distinct ids in [0, bq(t)], then -1
- *          padding (the output of hs_select_topk).  An id outside
- *          [-1, bq(t)] is skipped and reported as HS_ERR_INVALID_INDEX.
+ *          padding (the output of hs_select_topk).  An entry b >= 0 is used
+ *          when b <= bq(t) and b is larger than the entry before it; any
+ *          other non-negative entry is skipped and reported as
+ *          HS_ERR_INVALID_INDEX (the row's output is then unspecified).
  *   sink   [H] fp32 or NULL (NULL = no sink, i.e. -inf).
  *   out    [T, H, Dv] of `dtype`, contiguous, output.
  *   lse    [T, H] fp32, output.
