@@ -189,6 +189,29 @@ __device__ __forceinline__ bool rendezvous(Shared* sh, int wg, uint32_t& ph, lon
   return ok;
 }
 
+// NP K chunks (4 MMAs each, M=128 keys, N=64 heads, K=16) into S^T at d;
+// A = K panels 16 KB apart, B = Q chunks 8 KB apart.  No branch inside.
+template <int NP, bool FIRST>
+__device__ __forceinline__ void mma_run(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc) {
+#pragma unroll
+  for (int pn = 0; pn < NP; ++pn)
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      umma_ss(d, a0 + (uint64_t)((pn * kPanel) >> 4) + 2 * k,
+              b0 + (uint64_t)((pn * kQChunkBytes) >> 4) + 2 * k, idesc,
+              (FIRST && pn == 0 && k == 0) ? 0u : 1u);
+}
+
+// One 128-row dv chunk: O^T[c] (+)= V^T (MN-major, two 64-row panels) . P^T
+// over 128 keys = 8 MMAs (K=16 keys each, 16 key rows = 2 KB per step).
+template <bool FIRST>
+__device__ __forceinline__ void pv_run(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < kTile / 16; ++kk)
+    umma_ss(d, a0 + (uint64_t)(kk * 128), b0 + (uint64_t)(kk * 128), idesc,
+            (FIRST && kk == 0) ? 0u : 1u);
+}
+
 template <bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -329,26 +352,29 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           ph ^= 1;
         }
       };
-      // S^T(tile) = K_tile . Q^T into S buffer sidx & 1
+      // S^T(tile) = K_tile . Q^T into S buffer sidx & 1.  Each ring stage
+      // (two 64-column chunks) is one run of MMAs with no branch inside.
       auto qk = [&](bool last_tile) -> bool {
         const uint32_t buf = sidx & 1, use = sidx >> 1;
         if (!mbar_wait(&sh->sempty[buf], (use & 1) ^ 1, lim)) return false;
         tc_fence_after();
         const uint32_t d = tmem + kSCol + buf * kH;
         for (int s = 0; s < (p.nck + 1) / 2; ++s) {
-          if (!mbar_wait(&sh->full[slot], ph, lim)) return false;
-          tc_fence_after();
-          const int np = min(2, p.nck - 2 * s);
-          for (int pn = 0; pn < np; ++pn) {
-            const int c = 2 * s + pn;
-            if (!mbar_wait(&sh->qfull[c], qtok & 1, lim)) return false;
-            tc_fence_after();
-            const uint64_t a = ring_desc_k + (uint64_t)((slot * kSlotBytes + pn * kPanel) >> 4);
-            const uint64_t b = q_desc + (uint64_t)((c * kQChunkBytes) >> 4);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              umma_ss(d, a + 2 * k, b + 2 * k, id_qk, (c | k) != 0);
-            if (last_tile) umma_commit(&sh->qempty[c]);
+          const int c0 = 2 * s;
+          const bool two = c0 + 1 < p.nck;
+          if (!mbar_wait(&sh->full[slot], ph, lim)) return false;  // TMA stage
+          if (!mbar_wait(&sh->qfull[c0], qtok & 1, lim)) return false;
+          if (two && !mbar_wait(&sh->qfull[c0 + 1], qtok & 1, lim)) return false;
+          const uint64_t a = ring_desc_k + (uint64_t)((slot * kSlotBytes) >> 4);
+          const uint64_t b = q_desc + (uint64_t)((c0 * kQChunkBytes) >> 4);
+          if (s == 0) {
+            if (two) mma_run<2, true>(d, a, b, id_qk); else mma_run<1, true>(d, a, b, id_qk);
+          } else {
+            if (two) mma_run<2, false>(d, a, b, id_qk); else mma_run<1, false>(d, a, b, id_qk);
+          }
+          if (last_tile) {  // the token's last QK has read these Q chunks
+            umma_commit(&sh->qempty[c0]);
+            if (two) umma_commit(&sh->qempty[c0 + 1]);
           }
           umma_commit(&sh->empty[slot]);
           next_slot();
@@ -358,19 +384,16 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         issued = true;
         return true;
       };
-      // O^T += V_tile^T . P^T (waits for P of this tile)
+      // O^T += V_tile^T . P^T (waits for P of this tile); 8 MMAs per stage
       auto pv = [&](bool first_tile) -> bool {
         if (!mbar_wait(&sh->pfull, npv & 1, lim)) return false;
         tc_fence_after();
         for (int c = 0; c < p.nvc; ++c) {
-          if (!mbar_wait(&sh->full[slot], ph, lim)) return false;
-          tc_fence_after();
+          if (!mbar_wait(&sh->full[slot], ph, lim)) return false;  // TMA stage
           const uint64_t a0 = ring_desc_v + (uint64_t)((slot * kSlotBytes) >> 4);
           const uint32_t d = tmem + c * kH;
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ss(d, a0 + (uint64_t)(kk * 128), p_desc + (uint64_t)(kk * 128), id_pv,
-                    (!first_tile || kk > 0) ? 1u : 0u);
+          if (first_tile) pv_run<true>(d, a0, p_desc, id_pv);
+          else pv_run<false>(d, a0, p_desc, id_pv);
           umma_commit(&sh->empty[slot]);
           next_slot();
         }

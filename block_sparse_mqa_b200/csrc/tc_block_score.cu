@@ -14,15 +14,19 @@
 //    each); any remaining 64-column chunk (the RoPE part of Dk = 576) is a
 //    128-byte-swizzled shared-memory tile loaded by TMA (SS form).
 //  * Keys stream in tiles of 128 (always a whole number of blocks, starting
-//    at the document's first token) as 64-column K chunks through an 8-deep
-//    TMA ring of 16 KB stages; each chunk feeds four M=128, N=128, K=16 MMAs
-//    into one of two S accumulators in TMEM (double buffering lets the MMA
-//    run one key tile ahead of the softmax).
+//    at the document's first token) as 64-column K chunks (one 16 KB TMA box
+//    each); three chunks form one 48 KB stage of a 4-deep ring, so every
+//    pipeline wait of the MMA thread is followed by 12 M=128, N=128, K=16
+//    MMAs issued without a branch between them (a wait costs a few hundred
+//    cycles of issue and a branch between two MMAs about half the issue
+//    rate; both were measured).  The shared-memory (RoPE) chunk goes first.
+//    Each key tile accumulates into one of two S buffers in TMEM (double
+//    buffering lets the MMA run one key tile ahead of the softmax).
 //  * Softmax warps (thread = row) read S (tcgen05.ld), compute per-block
 //    log-sum-exp in the log2 domain with the block's own max (no underflow
 //    for far-below-max blocks) and keep the running row max and sum.  Block
-//    values go to a per-CTA global workspace slot [NBmax][128] (coalesced,
-//    L2 resident).  At the end of the tile each row has its LSE; the head
+//    values go to a per-CTA global workspace slot [2][NBmax][128] (coalesced,
+//    L2 resident; halves alternate by query tile).  At the end of the tile each row has its LSE; the head
 //    sum of exp2(blockLSE - LSE) is a 32-lane transpose-reduction per warp
 //    plus a fixed-order sum over the warps of a token (deterministic).
 //  * Warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner), warps 2-9
@@ -46,10 +50,12 @@ namespace {
 using namespace tc;
 
 constexpr int kThreads = 320;  // producer, MMA, 2 softmax warpgroups
-constexpr int kStages = 8;
 constexpr int kKeyTile = 128;
-constexpr int kStageBytes = kKeyTile * 64 * 2;  // 128 keys x 64 bf16
-constexpr int kMaxQhi = 2;                       // shared-memory Q chunks (Dk <= 640)
+constexpr int kChunkBytes = kKeyTile * 64 * 2;   // one TMA box: 128 keys x 64 bf16
+constexpr int kChunksPerStage = 3;               // 12 MMAs per pipeline wait
+constexpr int kStageBytes = kChunksPerStage * kChunkBytes;
+constexpr int kStages = 4;
+constexpr int kMaxQhi = 1;                       // shared-memory Q chunks (Dk <= 576)
 constexpr int kMaxTmemQ = 8;                     // TMEM Q chunks (first 512 columns)
 constexpr int kMaxDocs = 1024;
 constexpr int kSCol = 256;                       // S buffers at TMEM columns 256, 384
@@ -84,7 +90,8 @@ struct Shared {
   int abort_flag;
 };
 
-constexpr size_t kSmemBytes = 1024 + (size_t)(kStages + kMaxQhi) * kStageBytes + sizeof(Shared);
+constexpr size_t kSmemBytes =
+    1024 + (size_t)kStages * kStageBytes + (size_t)kMaxQhi * kChunkBytes + sizeof(Shared);
 
 struct Tile {
   int t0, tend, bos;
@@ -132,6 +139,27 @@ __device__ __forceinline__ float transpose_reduce_sum(float (&v)[32]) {
   return v[0];
 }
 
+// One ring stage = three 64-column K chunks = 12 MMAs (M=128, N=128, K=16)
+// into S accumulator d.  FIRST: the stage opens the S tile (its first MMA
+// overwrites d).  SS_FIRST: its first chunk is the shared-memory q chunk
+// (descriptor qd), the others come from TMEM q chunks tpos, tpos+1, ...
+template <bool FIRST, bool SS_FIRST>
+__device__ __forceinline__ void issue_stage(uint32_t d, uint32_t tmem, int tpos, uint64_t qd,
+                                            uint64_t b0, uint32_t idesc) {
+#pragma unroll
+  for (int c = 0; c < kChunksPerStage; ++c) {
+    const uint64_t bc = b0 + (uint64_t)((c * kChunkBytes) >> 4);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t acc = (FIRST && c == 0 && k == 0) ? 0u : 1u;
+      if (SS_FIRST && c == 0)
+        umma_ss(d, qd + 2 * k, bc + 2 * k, idesc, acc);
+      else
+        umma_ts(d, tmem + (uint32_t)((tpos + c) * 32 + k * 8), bc + 2 * k, idesc, acc);
+    }
+  }
+}
+
 template <int B>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -141,7 +169,7 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* stages = base;
   uint8_t* qhi = base + kStages * kStageBytes;
-  Shared* sh = reinterpret_cast<Shared*>(qhi + kMaxQhi * kStageBytes);
+  Shared* sh = reinterpret_cast<Shared*>(qhi + kMaxQhi * kChunkBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nd = p.num_docs;
 
@@ -212,22 +240,29 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
             give_up(sh, p.status);
             break;
           }
-          mbar_expect_tx(&sh->qhi_full, p.nq_smem * kStageBytes);
+          mbar_expect_tx(&sh->qhi_full, p.nq_smem * kChunkBytes);
           for (int j = 0; j < p.nq_smem; ++j)
-            tma_load_3d(qhi + j * kStageBytes, &qmap, &sh->qhi_full, (p.nq_tmem + j) * 64, 0,
+            tma_load_3d(qhi + j * kChunkBytes, &qmap, &sh->qhi_full, (p.nq_tmem + j) * 64, 0,
                         tl.t0);
           ++qfills;
         }
+        // per key tile, ring stages of three K chunks in the MMA's order: the
+        // shared-memory (RoPE) chunks first, then the TMEM chunks 0, 1, ...
         const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
+        const int spt = p.nck / kChunksPerStage;  // stages per key tile
         for (int kt = 0; kt < nkt && !aborted(sh); ++kt) {
-          for (int ch = 0; ch < p.nck; ++ch) {
+          for (int st = 0; st < spt; ++st) {
             if (!mbar_wait(&sh->kempty[kst], kph ^ 1, lim)) {
               give_up(sh, p.status);
               break;
             }
             mbar_expect_tx(&sh->kfull[kst], kStageBytes);
-            tma_load_2d(stages + kst * kStageBytes, &kmap, &sh->kfull[kst], ch * 64,
-                        tl.bos + kt * kKeyTile);
+            for (int j = 0; j < kChunksPerStage; ++j) {
+              const int pos = st * kChunksPerStage + j;
+              const int ch = pos < p.nq_smem ? p.nq_tmem + pos : pos - p.nq_smem;
+              tma_load_2d(stages + kst * kStageBytes + j * kChunkBytes, &kmap, &sh->kfull[kst],
+                          ch * 64, tl.bos + kt * kKeyTile);
+            }
             ++fills[kst];
             if (++kst == kStages) {
               kst = 0;
@@ -248,7 +283,7 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
       uint64_t qhi_desc[kMaxQhi];
 #pragma unroll
       for (int j = 0; j < kMaxQhi; ++j)
-        qhi_desc[j] = umma_desc_sw128(smem_u32(qhi + j * kStageBytes), 16, 1024);
+        qhi_desc[j] = umma_desc_sw128(smem_u32(qhi + j * kChunkBytes), 16, 1024);
       const uint64_t stage_desc0 = umma_desc_sw128(smem_u32(stages), 16, 1024);
       uint32_t kst = 0, kph = 0, sidx = 0;
       int qtile = 0;
@@ -263,8 +298,9 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
           give_up(sh, p.status);
           break;
         }
-        tc_fence_after();
+        tc_fence_after();  // q was written to TMEM by the softmax threads
         bool ok = true;
+        const int spt = p.nck / kChunksPerStage;
         for (int kt = 0; kt < nkt && ok; ++kt) {
           const uint32_t buf = sidx & 1, use = sidx >> 1;
           if (!mbar_wait(&sh->sempty[buf], (use & 1) ^ 1, lim)) {
@@ -273,22 +309,22 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
           }
           tc_fence_after();
           const uint32_t d = tmem + kSCol + buf * 128;
-          for (int ch = 0; ch < p.nck; ++ch) {
-            if (!mbar_wait(&sh->kfull[kst], kph, lim)) {
+          for (int st = 0; st < spt; ++st) {
+            if (!mbar_wait(&sh->kfull[kst], kph, lim)) {  // TMA stage (no fence needed)
               ok = false;
               break;
             }
-            tc_fence_after();
-            // stage descriptors advance by 16 KB = 1024 address units
-            const uint64_t bdesc = stage_desc0 + (uint64_t)(kst * (kStageBytes >> 4));
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint32_t accum = (ch | k) != 0;
-              if (ch < p.nq_tmem)
-                umma_ts(d, tmem + ch * 32 + k * 8, bdesc + 2 * k, idesc, accum);
-              else
-                umma_ss(d, qhi_desc[ch - p.nq_tmem] + 2 * k, bdesc + 2 * k, idesc, accum);
-            }
+            const uint64_t b0 = stage_desc0 + (uint64_t)((kst * kStageBytes) >> 4);
+            // 12 MMAs without a branch between them (a branch between two
+            // tcgen05.mma costs about half the issue rate); one stage pattern
+            // is chosen per stage
+            const int tpos = st * kChunksPerStage - p.nq_smem;  // first TMEM chunk
+            if (st == 0 && p.nq_smem > 0)
+              issue_stage<true, true>(d, tmem, tpos, qhi_desc[0], b0, idesc);
+            else if (st == 0)
+              issue_stage<true, false>(d, tmem, tpos, 0, b0, idesc);
+            else
+              issue_stage<false, false>(d, tmem, tpos, 0, b0, idesc);
             issued = true;
             umma_commit(&sh->kempty[kst]);
             if (++kst == kStages) {
@@ -323,7 +359,10 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
     const int H = p.H;
     const int hp = H / 32;  // warps per token
     const float sl2 = p.scale_log2;
-    float* const ws_row = p.ws + (size_t)blockIdx.x * p.nbmax * 128 + r;
+    // two workspace halves by query-tile parity: one warpgroup may already
+    // write the next tile's block values while the other still reads this
+    // tile's in its epilogue (they are never more than one tile apart)
+    float* const ws_cta = p.ws + (size_t)blockIdx.x * 2 * p.nbmax * 128 + r;
     uint32_t sbase = 0, all_ph = 0, wg_ph = 0;
     bool ok = true;
     // q rows of a tile into TMEM (this warpgroup's half of the chunks)
@@ -367,6 +406,7 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
       const int tok_c = valid ? tok : tl.tend - 1;
       const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
       float m = -INFINITY, l = 0.f;  // log2 domain
+      float* const ws_row = ws_cta + (size_t)(it & 1) * p.nbmax * 128;
       for (int kt = 0; kt < nkt; ++kt) {
         const uint32_t gs = sbase + kt;
         if ((int)(gs & 1) != wg) continue;
@@ -533,13 +573,14 @@ int grid_for(int total_tokens, int num_docs, int num_heads) {
 
 bool tc_block_score_supported(int num_heads, int dk, int block_size, int nbmax) {
   (void)nbmax;
-  return (num_heads == 32 || num_heads == 64 || num_heads == 128) && dk % 64 == 0 &&
-         dk >= 64 && dk <= 64 * (kMaxTmemQ + kMaxQhi) &&
+  // whole stages of three 64-column chunks: Dk in {192, 384, 576}
+  return (num_heads == 32 || num_heads == 64 || num_heads == 128) && dk % 192 == 0 &&
+         dk >= 192 && dk <= 64 * (kMaxTmemQ + kMaxQhi) &&
          (block_size == 16 || block_size == 32 || block_size == 64 || block_size == 128);
 }
 
 size_t tc_block_score_workspace(int total_tokens, int num_docs, int num_heads, int nbmax) {
-  return (size_t)grid_for(total_tokens, num_docs, num_heads) * nbmax * 128 * sizeof(float);
+  return (size_t)grid_for(total_tokens, num_docs, num_heads) * 2 * nbmax * 128 * sizeof(float);
 }
 
 // Data-dependent conditions of the tensor-core path (alignment, doc count).

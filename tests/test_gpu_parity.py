@@ -108,6 +108,22 @@ def test_block_window_variants(B, K, W):
     run_and_check(inp, B, K, W)
 
 
+@pytest.mark.parametrize("B,docs", [(16, [1000]), (32, [1300, 200])])
+def test_many_blocks_per_row(B, docs):
+    """More than 32 blocks per row with several query tiles per CTA: the
+    epilogue's block batches and the next tile's workspace writes overlap."""
+    inp = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=11)
+    run_and_check(inp, B, 6, 300)
+
+
+@pytest.mark.parametrize("H,dk,dv", [(32, 576, 512), (128, 192, 128)])
+def test_block_score_other_head_counts(H, dk, dv):
+    docs = [400, 150]
+    inp = _gpu_inputs(sum(docs), H, dk, dv, torch.bfloat16, docs, seed=12)
+    assert hs.path(hs.HS_OP_BLOCK_SCORE, torch.bfloat16, H, dk, dv, 64) == hs.HS_PATH_TCGEN05
+    run_and_check(inp, 64, 4, 100)
+
+
 def test_no_sink_and_large_sink():
     docs = [200, 77]
     inp = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=3)
