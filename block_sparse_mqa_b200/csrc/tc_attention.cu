@@ -261,48 +261,59 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // The whole warp issues: lane 0 waits for a free slot and arms its
+    // barrier with the stage's bytes, then the stage's TMA boxes are spread
+    // over the lanes (a single thread issues a box only every few hundred
+    // cycles, too slow for the per-block gather).
     if (lane == 0) {
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
       tma_prefetch_desc(&qmap);
-      int fills[kSlots], qfills[kMaxQChunks];
-      for (int s = 0; s < kSlots; ++s) fills[s] = 0;
-      for (int c = 0; c < kMaxQChunks; ++c) qfills[c] = 0;
-      uint32_t slot = 0, ph = 0;
-      bool stop = false;
-      // one ring stage: K (two 64-column chunks) or V (one 128-row dv chunk)
-      auto load_stage = [&](const TokenPlan& tp, int t, int tile, bool is_v, int idx2) -> bool {
-        if (!mbar_wait(&sh->empty[slot], ph ^ 1, lim)) return false;
-        const int npanel = is_v ? 2 : min(2, p.nck - 2 * idx2);
-        mbar_expect_tx(&sh->full[slot], npanel * kPanel);
-        uint8_t* dst = ring + slot * kSlotBytes;
-        for (int pn = 0; pn < npanel; ++pn) {
-          const int col = is_v ? (idx2 * 2 + pn) * 64 : (idx2 * 2 + pn) * 64;
-          for (int j = 0; j < per; ++j) {
-            int row0;
-            if (kSparse) {
-              const int slotn = tile * per + j;  // past the list: masked filler (own block)
-              const int b = slotn < tp.nsel ? sh->plist[slotn] : tp.bq;
-              row0 = tp.bos + b * p.B;
-            } else {
-              row0 = tp.wlo + tile * kTile;
-            }
-            tma_load_2d(dst + pn * kPanel + j * box_rows * 128, is_v ? &vmap : &kmap,
-                        &sh->full[slot], col, row0);
-          }
+    }
+    int fills[kSlots], qfills[kMaxQChunks];
+    for (int s = 0; s < kSlots; ++s) fills[s] = 0;
+    for (int c = 0; c < kMaxQChunks; ++c) qfills[c] = 0;
+    uint32_t slot = 0, ph = 0;
+    bool stop = false;
+    // one ring stage: K (two 64-column chunks) or V (one 128-row dv chunk)
+    auto load_stage = [&](const TokenPlan& tp, int tile, bool is_v, int idx2) -> bool {
+      const int npanel = is_v ? 2 : min(2, p.nck - 2 * idx2);
+      int ok = 1;
+      if (lane == 0) {
+        ok = mbar_wait(&sh->empty[slot], ph ^ 1, lim);
+        if (ok) mbar_expect_tx(&sh->full[slot], npanel * kPanel);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) return false;
+      __syncwarp();
+      uint8_t* dst = ring + slot * kSlotBytes;
+      for (int bx = lane; bx < npanel * per; bx += 32) {
+        const int pn = bx / per, j = bx - pn * per;
+        const int col = (idx2 * 2 + pn) * 64;
+        int row0;
+        if (kSparse) {
+          const int slotn = tile * per + j;  // past the list: masked filler (own block)
+          const int b = slotn < tp.nsel ? sh->plist[slotn] : tp.bq;
+          row0 = tp.bos + b * p.B;
+        } else {
+          row0 = tp.wlo + tile * kTile;
         }
-        ++fills[slot];
-        if (++slot == kSlots) {
-          slot = 0;
-          ph ^= 1;
-        }
-        return true;
-      };
-      const int nks = (p.nck + 1) / 2;  // K stages per tile
-      for (int t = blockIdx.x; t < p.T && !stop; t += G) {
-        const TokenPlan tp = plan_token<kSparse>(p, t, true);
-        if (!tp.ok || tp.ntile == 0) continue;
-        if (kSparse) {  // this token's selected blocks, once
+        tma_load_2d(dst + pn * kPanel + j * box_rows * 128, is_v ? &vmap : &kmap,
+                    &sh->full[slot], col, row0);
+      }
+      ++fills[slot];
+      if (++slot == kSlots) {
+        slot = 0;
+        ph ^= 1;
+      }
+      return true;
+    };
+    const int nks = (p.nck + 1) / 2;  // K stages per tile
+    for (int t = blockIdx.x; t < p.T && !stop; t += G) {
+      const TokenPlan tp = plan_token<kSparse>(p, t, lane == 0);
+      if (!tp.ok || tp.ntile == 0) continue;
+      if (kSparse) {  // this token's selected blocks, once
+        if (lane == 0) {
           const int32_t* row = p.idx + (int64_t)t * p.topk;
           int n = 0;
           for (int s2 = 0; s2 < p.topk; ++s2) {
@@ -310,30 +321,39 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
             if (entry_ok(row, s2, tp.bq, b)) sh->plist[n++] = b;
           }
         }
-        // Q_t chunks, each as soon as the previous token's last QK released it
-        for (int c = 0; c < p.nck; ++c) {
-          if (qfills[c] > 0 && !mbar_wait(&sh->qempty[c], (qfills[c] - 1) & 1, lim)) {
-            stop = true;
-            break;
-          }
+        __syncwarp();
+      }
+      // Q_t chunks (lane c loads chunk c), each as soon as the previous
+      // token's last QK released it
+      int qok = 1;
+      if (lane < p.nck) {
+        const int c = lane;
+        if (qfills[c] > 0) qok = mbar_wait(&sh->qempty[c], (qfills[c] - 1) & 1, lim);
+        if (qok) {
           mbar_expect_tx(&sh->qfull[c], kQChunkBytes);
           tma_load_3d(qbuf + c * kQChunkBytes, &qmap, &sh->qfull[c], c * 64, 0, t);
           ++qfills[c];
         }
-        if (stop) break;
-        for (int s = 0; s < nks && !stop; ++s) stop = !load_stage(tp, t, 0, false, s);
-        for (int i = 0; i < tp.ntile && !stop; ++i) {
-          if (i + 1 < tp.ntile)
-            for (int s = 0; s < nks && !stop; ++s) stop = !load_stage(tp, t, i + 1, false, s);
-          for (int c = 0; c < p.nvc && !stop; ++c) stop = !load_stage(tp, t, i, true, c);
-        }
       }
-      if (stop) give_up(sh, p.status);
+      if (!__all_sync(0xffffffffu, qok)) {
+        stop = true;
+        break;
+      }
+      for (int s = 0; s < nks && !stop; ++s) stop = !load_stage(tp, 0, false, s);
+      for (int i = 0; i < tp.ntile && !stop; ++i) {
+        if (i + 1 < tp.ntile)
+          for (int s = 0; s < nks && !stop; ++s) stop = !load_stage(tp, i + 1, false, s);
+        for (int c = 0; c < p.nvc && !stop; ++c) stop = !load_stage(tp, i, true, c);
+      }
+      __syncwarp();  // plist is rewritten for the next token only after all lanes used it
+    }
+    if (stop && lane == 0) give_up(sh, p.status);
+    // no copy may still be landing when the CTA exits
+    if (lane == 0)
       for (int s = 0; s < kSlots; ++s)
         if (fills[s] > 0) mbar_wait(&sh->full[s], (fills[s] - 1) & 1, kDefaultWaitNs);
-      for (int c = 0; c < kMaxQChunks; ++c)
-        if (qfills[c] > 0) mbar_wait(&sh->qfull[c], (qfills[c] - 1) & 1, kDefaultWaitNs);
-    }
+    if (lane < p.nck && qfills[lane] > 0)
+      mbar_wait(&sh->qfull[lane], (qfills[lane] - 1) & 1, kDefaultWaitNs);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -354,17 +374,19 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       };
       // S^T(tile) = K_tile . Q^T into S buffer sidx & 1.  Each ring stage
       // (two 64-column chunks) is one run of MMAs with no branch inside.
-      auto qk = [&](bool last_tile) -> bool {
+      auto qk = [&](bool first_tile, bool last_tile) -> bool {
         const uint32_t buf = sidx & 1, use = sidx >> 1;
-        if (!mbar_wait(&sh->sempty[buf], (use & 1) ^ 1, lim)) return false;
+        if (!mbar_wait_spin(&sh->sempty[buf], (use & 1) ^ 1, lim)) return false;
         tc_fence_after();
         const uint32_t d = tmem + kSCol + buf * kH;
         for (int s = 0; s < (p.nck + 1) / 2; ++s) {
           const int c0 = 2 * s;
           const bool two = c0 + 1 < p.nck;
-          if (!mbar_wait(&sh->full[slot], ph, lim)) return false;  // TMA stage
-          if (!mbar_wait(&sh->qfull[c0], qtok & 1, lim)) return false;
-          if (two && !mbar_wait(&sh->qfull[c0 + 1], qtok & 1, lim)) return false;
+          if (!mbar_wait_spin(&sh->full[slot], ph, lim)) return false;  // TMA stage
+          if (first_tile) {  // the token's q chunks (resident for all its tiles)
+            if (!mbar_wait_spin(&sh->qfull[c0], qtok & 1, lim)) return false;
+            if (two && !mbar_wait_spin(&sh->qfull[c0 + 1], qtok & 1, lim)) return false;
+          }
           const uint64_t a = ring_desc_k + (uint64_t)((slot * kSlotBytes) >> 4);
           const uint64_t b = q_desc + (uint64_t)((c0 * kQChunkBytes) >> 4);
           if (s == 0) {
@@ -386,10 +408,10 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       };
       // O^T += V_tile^T . P^T (waits for P of this tile); 8 MMAs per stage
       auto pv = [&](bool first_tile) -> bool {
-        if (!mbar_wait(&sh->pfull, npv & 1, lim)) return false;
+        if (!mbar_wait_spin(&sh->pfull, npv & 1, lim)) return false;
         tc_fence_after();
         for (int c = 0; c < p.nvc; ++c) {
-          if (!mbar_wait(&sh->full[slot], ph, lim)) return false;  // TMA stage
+          if (!mbar_wait_spin(&sh->full[slot], ph, lim)) return false;  // TMA stage
           const uint64_t a0 = ring_desc_v + (uint64_t)((slot * kSlotBytes) >> 4);
           const uint32_t d = tmem + c * kH;
           if (first_tile) pv_run<true>(d, a0, p_desc, id_pv);
@@ -404,12 +426,12 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       for (int t = blockIdx.x; t < p.T && !stop; t += G) {
         const TokenPlan tp = plan_token<kSparse>(p, t, false);
         if (!tp.ok || tp.ntile == 0) continue;
-        if (!qk(tp.ntile == 1)) { stop = true; break; }
+        if (!qk(true, tp.ntile == 1)) { stop = true; break; }
         // O^T of the previous token must have been read out before PV(0)
         if (ntok > 0 && !mbar_wait(&sh->oempty, (ntok - 1) & 1, lim)) { stop = true; break; }
         tc_fence_after();
         for (int i = 0; i < tp.ntile; ++i) {
-          if (i + 1 < tp.ntile && !qk(i + 2 == tp.ntile)) { stop = true; break; }
+          if (i + 1 < tp.ntile && !qk(false, i + 2 == tp.ntile)) { stop = true; break; }
           if (!pv(i == 0)) { stop = true; break; }
         }
         if (stop) break;

@@ -303,14 +303,14 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
         const int spt = p.nck / kChunksPerStage;
         for (int kt = 0; kt < nkt && ok; ++kt) {
           const uint32_t buf = sidx & 1, use = sidx >> 1;
-          if (!mbar_wait(&sh->sempty[buf], (use & 1) ^ 1, lim)) {
+          if (!mbar_wait_spin(&sh->sempty[buf], (use & 1) ^ 1, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t d = tmem + kSCol + buf * 128;
           for (int st = 0; st < spt; ++st) {
-            if (!mbar_wait(&sh->kfull[kst], kph, lim)) {  // TMA stage (no fence needed)
+            if (!mbar_wait_spin(&sh->kfull[kst], kph, lim)) {  // TMA stage (no fence needed)
               ok = false;
               break;
             }

@@ -71,6 +71,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
   }
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait variant for the single MMA-issuing thread: the non-suspending
+// test_wait is cheaper than try_wait when the phase has usually completed
+// already (it was measured to cost fewer issue cycles); same bound.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity,
+                                               long long limit_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return mbar_wait(bar, parity, limit_ns);
+}
+
 // Default limit of every pipeline wait: two seconds.
 constexpr long long kDefaultWaitNs = 2000000000ll;
 
