@@ -46,15 +46,30 @@ UNIT = "tokens/s"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=workloads.MAIN.name)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=48,
+    ap.add_argument("--cpu-rows", type=int, default=1536,
                     help="query rows of the oracle sample (cpu_baseline / reference arm)")
     return ap.parse_args()
+
+
+def ncu_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu record, or
+    None when the kernel source changed since the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        rec = json.load(open(p))[kernel]
+        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    except (OSError, KeyError, ValueError):
+        return None
+    if hashlib.sha256(src).hexdigest() != rec["sha256"]:
+        return None
+    return rec["bytes"]
 
 
 def peaks():
@@ -117,7 +132,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -231,12 +246,21 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a host scalar over all ranks (the device-timed region of the
+    slowest rank defines the job's time)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens(tokens_per_rank, world):
+    """Whole-job units: every rank processes its own replica of the workload
+    (independent documents, no data-path collective)."""
+    return tokens_per_rank * world
 
 
 # ---------------------------------------------------------------------------
@@ -326,7 +350,7 @@ def run_ours(args, wl, world, rank):
     step_ms = [sum(per_phase[p][s] for p in range(nph)) for s in range(args.steps)]
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
-    tokens = wl.total_tokens * world
+    tokens = job_tokens(wl.total_tokens, world)
     value = tokens / (ms_per_step / 1e3)
 
     pk = peaks()
@@ -353,7 +377,8 @@ def run_ours(args, wl, world, rank):
     dom = max(("score", "sparse", "swa"), key=lambda ph: avg[ph])
     roof = {"bound": "tensor", "achieved": kernels[dom]["tflops"], "peak": pk["bf16_tflops"],
             "unit": "TFLOP/s", "frac": kernels[dom]["tflops"] / pk["bf16_tflops"],
-            "traffic": None, "kernel": dom,
+            "traffic": ncu_traffic(dom) if wl.name == workloads.MAIN.name else None,
+            "kernel": dom,
             "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % pk["source"]}
     contraction_tflops = (flops["score"] + flops["sparse"] + flops["swa"]) / (
         (avg["score"] + avg["sparse"] + avg["swa"]) / 1e3) / 1e12

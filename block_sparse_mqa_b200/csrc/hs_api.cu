@@ -25,7 +25,7 @@ int* g_status_ptr[kMaxDevices];
 std::mutex g_status_mu;
 
 std::atomic<int> g_force_simt{0};
-std::atomic<long long> g_wait_limit{0};
+std::atomic<long long> g_wait_limit{0};  // 0 = the kernels' default bound
 
 thread_local char g_last_error[512];
 
@@ -139,7 +139,14 @@ const char* hs_last_error(void) { return g_last_error; }
 
 void hs_set_force_simt(int on) { g_force_simt.store(on ? 1 : 0); }
 
-void hs_set_wait_limit(long long iterations) { g_wait_limit.store(iterations > 0 ? iterations : 0); }
+hs_status hs_selftest_wait(long long limit_ns, hs_stream_t stream) {
+  if (limit_ns < 1 || limit_ns > 1000000000ll)
+    return fail(HS_ERR_INVALID_ARG, "limit_ns %lld not in [1, 1e9]", limit_ns);
+  int* st = nullptr;
+  hs_status r = status_ptr(&st);
+  if (r != HS_OK) return r;
+  return launched(hs::launch_selftest_wait(limit_ns, st, stream), "self-test wait");
+}
 
 int hs_path(int op, hs_dtype dtype, int num_heads, int dk, int dv, int block_size) {
   if (dtype != HS_F32 && dtype != HS_BF16) return -1;

@@ -65,4 +65,7 @@ bool tc_attention_eligible(const AttnArgs& a);  // alignment conditions
 cudaError_t launch_tc_attention(const AttnArgs& a, bool sparse, long long wait_limit,
                                 cudaStream_t s);
 
+// One thread waits (bounded) on an mbarrier nothing arrives at.
+cudaError_t launch_selftest_wait(long long limit_ns, int* status, cudaStream_t s);
+
 }  // namespace hs

@@ -43,7 +43,7 @@ HS_PATH_TCGEN05 = 1
 EXPORTS = (
     "hs_block_score", "hs_select_topk", "hs_sparse_mqa_fwd", "hs_swa_mqa_fwd",
     "hs_workspace_size", "hs_path", "hs_poll_status", "hs_set_force_simt",
-    "hs_set_wait_limit", "hs_status_string", "hs_last_error", "hs_version",
+    "hs_selftest_wait", "hs_status_string", "hs_last_error", "hs_version",
 )
 
 
@@ -84,8 +84,8 @@ def lib() -> ctypes.CDLL:
     L.hs_poll_status.argtypes = [_vp]
     L.hs_set_force_simt.argtypes = [_int]
     L.hs_set_force_simt.restype = None
-    L.hs_set_wait_limit.argtypes = [ctypes.c_longlong]
-    L.hs_set_wait_limit.restype = None
+    L.hs_selftest_wait.argtypes = [ctypes.c_longlong, _vp]
+    L.hs_selftest_wait.restype = _int
     L.hs_status_string.argtypes = [_int]
     L.hs_status_string.restype = ctypes.c_char_p
     L.hs_last_error.argtypes = []
@@ -143,8 +143,10 @@ def set_force_simt(on: bool):
     lib().hs_set_force_simt(1 if on else 0)
 
 
-def set_wait_limit(iterations: int):
-    lib().hs_set_wait_limit(int(iterations))
+def selftest_wait(limit_ns: int, device=None):
+    """Launch the bounded-wait self test (see include/hs.h)."""
+    dev = torch.device("cuda" if device is None else device)
+    _check(lib().hs_selftest_wait(int(limit_ns), _stream(dev)))
 
 
 def path(op: int, dtype: torch.dtype, num_heads: int, dk: int, dv: int, block_size: int) -> int:

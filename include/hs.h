@@ -220,10 +220,13 @@ hs_status hs_poll_status(hs_stream_t stream);
  * where a tensor-core kernel exists.  Process-wide; not for production. */
 void hs_set_force_simt(int on);
 
-/* Testing aid: overrides the iteration limit of the tensor-core kernels'
- * pipeline waits (0 restores the default).  A tiny limit makes the waits
- * give up early and report HS_ERR_TIMEOUT instead of computing. */
-void hs_set_wait_limit(long long iterations);
+/* Failure-detection self test (no counterpart in the method): launches one
+ * thread that waits on an mbarrier nothing will ever arrive at, with the
+ * same bounded-wait routine the tensor-core pipelines use and a limit of
+ * limit_ns nanoseconds (1 .. 10^9).  The wait gives up, the kernel records
+ * HS_ERR_TIMEOUT in the device status word and returns normally; the next
+ * hs_poll_status() reports it.  Nothing is in flight when it gives up. */
+hs_status hs_selftest_wait(long long limit_ns, hs_stream_t stream);
 
 const char* hs_status_string(hs_status status);
 

@@ -116,3 +116,9 @@ def test_binding_refuses_cpu_tensors():
     cu = torch.tensor([0, 4], dtype=torch.int32)
     with pytest.raises(ValueError):
         hs.hs_block_score(q, k, cu, 4, 16)
+
+
+def test_selftest_rejects_bad_limit():
+    L = hs.lib()
+    assert L.hs_selftest_wait(0, None) == hs.HS_ERR_INVALID_ARG
+    assert L.hs_selftest_wait(10**10, None) == hs.HS_ERR_INVALID_ARG
