@@ -118,6 +118,12 @@ hs_status launched(cudaError_t e, const char* what) {
 
 }  // namespace
 
+namespace hs {
+// Lets other translation units of the library report a host-side failure
+// through hs_last_error().
+hs_status report_error(hs_status st, const char* msg) { return fail(st, "%s", msg); }
+}  // namespace hs
+
 extern "C" {
 
 int hs_version(void) { return 100; }

@@ -65,6 +65,9 @@ bool tc_attention_eligible(const AttnArgs& a);  // alignment conditions
 cudaError_t launch_tc_attention(const AttnArgs& a, bool sparse, long long wait_limit,
                                 cudaStream_t s);
 
+// Records msg as the calling thread's hs_last_error() and returns st.
+hs_status report_error(hs_status st, const char* msg);
+
 // One thread waits (bounded) on an mbarrier nothing arrives at.
 cudaError_t launch_selftest_wait(long long limit_ns, int* status, cudaStream_t s);
 

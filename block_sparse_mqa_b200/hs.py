@@ -44,6 +44,7 @@ EXPORTS = (
     "hs_block_score", "hs_select_topk", "hs_sparse_mqa_fwd", "hs_swa_mqa_fwd",
     "hs_workspace_size", "hs_path", "hs_poll_status", "hs_set_force_simt",
     "hs_selftest_wait", "hs_status_string", "hs_last_error", "hs_version",
+    "hs_block_score_static",
 )
 
 
@@ -72,6 +73,8 @@ def lib() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     L.hs_block_score.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _int, _int, _int, _int, _int,
                                  _int, _flt, _int, _vp, _vp, _int, _vp, _vp, _szt, _vp]
+    L.hs_block_score_static.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _int, _int, _int, _int,
+                                        _int, _int, _flt, _int, _vp, _vp, _int, _vp, _vp]
     L.hs_select_topk.argtypes = [_vp, _int, _vp, _int, _int, _int, _int, _int, _vp, _vp]
     L.hs_sparse_mqa_fwd.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _int, _int, _int,
                                     _int, _int, _int, _int, _flt, _vp, _int, _int, _vp, _vp, _vp,
@@ -91,7 +94,7 @@ def lib() -> ctypes.CDLL:
     L.hs_last_error.argtypes = []
     L.hs_last_error.restype = ctypes.c_char_p
     for fn in ("hs_block_score", "hs_select_topk", "hs_sparse_mqa_fwd", "hs_swa_mqa_fwd",
-               "hs_poll_status"):
+               "hs_poll_status", "hs_block_score_static"):
         getattr(L, fn).restype = _int
     _lib = L
     return L
@@ -193,6 +196,28 @@ def hs_block_score(q, k, cu_seqlens, max_seqlen: int, block_size: int,
         _ptr(q), qrs, qhs, _ptr(k), krs, _ptr(cu_seqlens), nd, T, int(max_seqlen), H, Dk,
         _dtype_code(q), float(softmax_scale), int(block_size), _ptr(lse), _ptr(bs), bs.stride(0),
         _ptr(blse), _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(dev)))
+    return lse, bs, blse
+
+
+def hs_block_score_static(q, k, cu_seqlens, max_seqlen: int, block_size: int,
+                          softmax_scale: float = 0.0, want_block_lse: bool = False):
+    """Step 1 without a workspace: for callers that cannot allocate device
+    memory, the library's fixed 16 MiB scratch array is used instead (see
+    include/hs.h for the size limit and the one-call-at-a-time rule).  The
+    output tensors here are allocated by torch for convenience; a caller that
+    cannot allocate passes its own output pointers to the C entry point."""
+    _need_cuda(q, k, cu_seqlens)
+    qrs, qhs, krs = _qk_strides(q, k)
+    T, H, Dk = q.shape
+    nb = nbmax(max_seqlen, block_size)
+    dev = q.device
+    lse = torch.empty((T, H), device=dev, dtype=torch.float32)
+    bs = torch.empty((T, nb), device=dev, dtype=torch.float32)
+    blse = torch.empty((T, H, nb), device=dev, dtype=torch.float32) if want_block_lse else None
+    _check(lib().hs_block_score_static(
+        _ptr(q), qrs, qhs, _ptr(k), krs, _ptr(cu_seqlens), cu_seqlens.numel() - 1, T,
+        int(max_seqlen), H, Dk, _dtype_code(q), float(softmax_scale), int(block_size), _ptr(lse),
+        _ptr(bs), bs.stride(0), _ptr(blse), _stream(dev)))
     return lse, bs, blse
 
 

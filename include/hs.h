@@ -200,6 +200,41 @@ hs_status hs_swa_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_str
                          float softmax_scale, int window, const float* sink,
                          void* out, float* lse, hs_stream_t stream);
 
+/*
+ * Step 1 for callers that cannot allocate device memory.
+ * The method has no counterpart of this call; it is a deployment aid.
+ *
+ * hs_block_score needs a caller-provided workspace.  Some callers cannot
+ * allocate one: code running where an allocator call is not allowed (inside
+ * a framework's kernel-launch hook, a real-time loop that must not take the
+ * allocator's locks or synchronisation, a process whose device memory is
+ * fixed up front).  This call computes exactly what hs_block_score computes,
+ * with the same arguments minus the workspace, and takes its scratch from a
+ * 16 MiB array in the library's own device memory (every GPU on which the
+ * library is loaded holds that array until the process exits).  It calls no
+ * allocation or free routine.
+ *
+ *   - Problems whose scratch would exceed 16 MiB (hs_workspace_size of
+ *     HS_OP_BLOCK_SCORE > 16 MiB; with 148 SMs that is about 110 key blocks
+ *     per document, e.g. max_seqlen 7040 at block size 64) are rejected on
+ *     the host with HS_ERR_WORKSPACE before any device work; use
+ *     hs_block_score with a workspace for them.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) while that device is current; make that first
+ *     call before any stream capture.
+ *   - All calls share the one array and nothing is cleared between calls
+ *     (no scratch value is read before the kernel writes it, so the previous
+ *     contents do not matter).  Calls that may overlap on the GPU (other
+ *     streams, other host threads) race on the array: serialise them.
+ */
+hs_status hs_block_score_static(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                                const void* k, int64_t k_row_stride,
+                                const int32_t* cu_seqlens, int num_docs, int total_tokens,
+                                int max_seqlen, int num_heads, int dk, hs_dtype dtype,
+                                float softmax_scale, int block_size,
+                                float* lse, float* block_score, int nb_stride, float* block_lse,
+                                hs_stream_t stream);
+
 /* ---------------------------------------------------------------- helpers */
 
 /* Bytes of `workspace` that op needs for these sizes (0 = none).  Only
