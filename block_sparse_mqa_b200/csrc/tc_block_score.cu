@@ -10,9 +10,10 @@
 //  * A query tile is 128 rows = (128 / H) consecutive tokens x H heads of one
 //    document; q[T, H, Dk] rows are (token, head) pairs, so a tile is a
 //    plain 128-row slab.  The first min(Dk, 512) columns of the tile live in
-//    TMEM as the A operand (TS form: written by the softmax threads, one row
-//    each); any remaining 64-column chunk (the RoPE part of Dk = 576) is a
-//    128-byte-swizzled shared-memory tile loaded by TMA (SS form).
+//    TMEM as the A operand (TS form): TMA brings them through the ring and
+//    the MMA thread copies them into TMEM with tcgen05.cp (the same swizzled
+//    K-major slabs an SS MMA would read); any remaining 64-column chunk (the
+//    RoPE part of Dk = 576) stays a shared-memory tile (SS form).
 //  * Keys stream in tiles of 128 (always a whole number of blocks, starting
 //    at the document's first token) as 64-column K chunks (one 16 KB TMA box
 //    each); three chunks form one 48 KB stage of a 4-deep ring, so every
@@ -31,7 +32,7 @@
 //    plus a fixed-order sum over the warps of a token (deterministic).
 //  * Warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner), warps 2-9
 //    = two softmax warpgroups that take alternate S tiles (one S buffer
-//    each), load q into TMEM and share the epilogue.  Per-row running
+//    each) and share the epilogue.  Per-row running
 //    (max, sum) pairs of the two warpgroups are merged at the end of the
 //    tile; S is read in 32-column chunks with the next tcgen05.ld in flight.
 //    Every wait is bounded; a timeout records HS_ERR_TIMEOUT, drains
@@ -79,7 +80,7 @@ struct BSParams {
 
 struct Shared {
   uint64_t kfull[kStages], kempty[kStages];
-  uint64_t qhi_full, qhi_empty, qlo_full, drain;
+  uint64_t qhi_full, qhi_empty, qdone, drain;  // qdone: a tile's MMAs have completed
   uint64_t sfull[2], sempty[2];
   uint64_t epi_all;    // rendezvous of both softmax warpgroups (256 threads)
   uint64_t epi_wg[2];  // rendezvous inside one warpgroup (128 threads)
@@ -180,7 +181,7 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
     }
     mbar_init(&sh->qhi_full, 1);
     mbar_init(&sh->qhi_empty, 1);
-    mbar_init(&sh->qlo_full, 256);
+    mbar_init(&sh->qdone, 1);
     mbar_init(&sh->drain, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->sfull[b], 1);
@@ -246,6 +247,24 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
                         tl.t0);
           ++qfills;
         }
+        // the tile's q chunks that live in TMEM pass through the ring (three
+        // per stage); the MMA thread copies them into TMEM with tcgen05.cp
+        for (int q0 = 0; q0 < p.nq_tmem && !aborted(sh); q0 += kChunksPerStage) {
+          const int n = min(kChunksPerStage, p.nq_tmem - q0);
+          if (!mbar_wait(&sh->kempty[kst], kph ^ 1, lim)) {
+            give_up(sh, p.status);
+            break;
+          }
+          mbar_expect_tx(&sh->kfull[kst], n * kChunkBytes);
+          for (int j = 0; j < n; ++j)
+            tma_load_3d(stages + kst * kStageBytes + j * kChunkBytes, &qmap, &sh->kfull[kst],
+                        (q0 + j) * 64, 0, tl.t0);
+          ++fills[kst];
+          if (++kst == kStages) {
+            kst = 0;
+            kph ^= 1;
+          }
+        }
         // per key tile, ring stages of three K chunks in the MMA's order: the
         // shared-memory (RoPE) chunks first, then the TMEM chunks 0, 1, ...
         const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
@@ -293,13 +312,33 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
         if (g >= total) continue;
         const Tile tl = tile_of(g, sh->prefix, nd, p.cu, p.tpt);
         const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
-        if (!mbar_wait(&sh->qlo_full, qtile & 1, lim) ||
+        // q enters TMEM by tcgen05.cp from the ring, once every MMA of the
+        // previous tile (which read the old q) has completed
+        if ((qtile > 0 && !mbar_wait_spin(&sh->qdone, (qtile - 1) & 1, lim)) ||
             (p.nq_smem > 0 && !mbar_wait(&sh->qhi_full, qtile & 1, lim))) {
           give_up(sh, p.status);
           break;
         }
-        tc_fence_after();  // q was written to TMEM by the softmax threads
+        tc_fence_after();
         bool ok = true;
+        for (int q0 = 0; q0 < p.nq_tmem; q0 += kChunksPerStage) {
+          const int n = min(kChunksPerStage, p.nq_tmem - q0);
+          if (!mbar_wait_spin(&sh->kfull[kst], kph, lim)) {  // TMA stage
+            ok = false;
+            break;
+          }
+          const uint64_t b0 = stage_desc0 + (uint64_t)((kst * kStageBytes) >> 4);
+          for (int j = 0; j < n; ++j)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)  // 128 rows x 16 elements per copy
+              tmem_cp_128x256b(tmem + (uint32_t)((q0 + j) * 32 + k * 8),
+                               b0 + (uint64_t)((j * kChunkBytes) >> 4) + 2 * k);
+          umma_commit(&sh->kempty[kst]);  // the copies have read the stage
+          if (++kst == kStages) {
+            kst = 0;
+            kph ^= 1;
+          }
+        }
         const int spt = p.nck / kChunksPerStage;
         for (int kt = 0; kt < nkt && ok; ++kt) {
           const uint32_t buf = sidx & 1, use = sidx >> 1;
@@ -341,6 +380,7 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
           break;
         }
         if (p.nq_smem > 0) umma_commit(&sh->qhi_empty);
+        umma_commit(&sh->qdone);
         ++qtile;
       }
       if (issued) {  // every MMA done before TMEM is released
@@ -365,29 +405,6 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
     float* const ws_cta = p.ws + (size_t)blockIdx.x * 2 * p.nbmax * 128 + r;
     uint32_t sbase = 0, all_ph = 0, wg_ph = 0;
     bool ok = true;
-    // q rows of a tile into TMEM (this warpgroup's half of the chunks)
-    auto load_qlo = [&](const Tile& tq) {
-      const int tk = min(tq.t0 + r / H, tq.tend - 1);
-      const __nv_bfloat16* src = p.q + (int64_t)tk * p.qrs + (int64_t)(r % H) * p.qhs;
-      const int half = (p.nq_tmem + 1) >> 1;
-      const int c0 = wg ? half : 0, c1 = wg ? p.nq_tmem : half;
-      for (int ch = c0; ch < c1; ++ch) {
-        uint32_t v[32];
-        const uint4* s4 = reinterpret_cast<const uint4*>(src + ch * 64);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 x = __ldg(s4 + i);
-          v[4 * i + 0] = x.x;
-          v[4 * i + 1] = x.y;
-          v[4 * i + 2] = x.z;
-          v[4 * i + 3] = x.w;
-        }
-        tmem_st32(lane_base + ch * 32, v);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&sh->qlo_full);
-    };
     auto tile_at = [&](int it2, Tile& out) -> bool {
       if (it2 * G >= total) return false;
       const int g2 = it2 * G + ((it2 & 1) ? (G - 1 - cta) : cta);
@@ -397,7 +414,6 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
     };
     Tile cur;
     bool have = tile_at(0, cur);
-    if (have) load_qlo(cur);
     for (int it = 0; have && ok && !aborted(sh); ++it) {
       const Tile tl = cur;
       const int tok = tl.t0 + r / H;
@@ -513,9 +529,7 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
                       (m1 == -INFINITY ? 0.f : l1 * fast_exp2(m1 - M));
       const float lse2 = M + fast_log2(L);
       if (wg == 0 && valid) p.lse[(int64_t)tok * H + h] = lse2 * kLn2;
-      // every MMA of this tile is complete: the next tile's q may enter TMEM
       have = tile_at(it + 1, cur);
-      if (have) load_qlo(cur);
       // ---- head-summed block masses (and optional per-head block LSE)
       const int bq = valid ? (tok - tl.bos) / B : -1;
       float* blo = (valid && p.block_lse) ? p.block_lse + ((int64_t)tok * H + h) * p.nbs : nullptr;

@@ -255,6 +255,14 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       : "memory");
 }
 
+// Asynchronous copy of a 128-row x 256-bit slab from shared memory (matrix
+// descriptor, same format as an MMA operand) into TMEM lanes 0..127, eight
+// 32-bit columns from taddr.  Ordered before later tcgen05.mma of the same
+// thread.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive on `bar` once every previously issued tcgen05.mma of this thread
 // has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
