@@ -55,6 +55,7 @@ from typing import Optional
 import numpy as np
 
 __all__ = [
+    "RowSubset",
     "doc_bounds",
     "num_blocks",
     "block_score",
@@ -115,7 +116,22 @@ def _scale(scale: Optional[float], dk: int) -> float:
 
 
 def _f64(x) -> np.ndarray:
+    if isinstance(x, RowSubset):
+        return x
     return np.asarray(x, dtype=np.float64)
+
+
+class RowSubset:
+    """q given only for some query tokens (sampled checks at sizes where a
+    full float64 copy of q would not fit in host memory).  Indexing by a
+    token returns its [H, Dk] float64 row; other tokens are absent."""
+
+    def __init__(self, rows: dict, shape):
+        self._rows = {int(t): np.asarray(v, dtype=np.float64) for t, v in rows.items()}
+        self.shape = tuple(shape)
+
+    def __getitem__(self, t):
+        return self._rows[int(t)]
 
 
 # ---------------------------------------------------------------------------

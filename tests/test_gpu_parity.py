@@ -24,9 +24,15 @@ def _gpu_inputs(T, H, dk, dv, dtype, docs, seed=0, sink_std=1.0):
                              sink_std=sink_std)
 
 
-def _host(inp):
+def _host(inp, rows=None):
     f = lambda t: t.detach().cpu().double().numpy()
-    return f(inp.q), f(inp.k), f(inp.v), f(inp.sink), inp.cu_seqlens.cpu().tolist()
+    if rows is not None and inp.q.numel() > (1 << 27):  # only the sampled q rows
+        rr = torch.as_tensor(np.asarray(rows), device=inp.q.device)
+        qs = f(inp.q[rr])
+        q = O.RowSubset({int(t): qs[i] for i, t in enumerate(rows)}, inp.q.shape)
+    else:
+        q = f(inp.q)
+    return q, f(inp.k), f(inp.v), f(inp.sink), inp.cu_seqlens.cpu().tolist()
 
 
 def _expect_path(op, inp, B):
@@ -37,7 +43,7 @@ def run_and_check(inp, B, K, W, rows=None, sink=True, scale=0.0, v=None, check_p
     """Run the four steps on the GPU and compare each against the oracle
     (stage-isolated: the oracle's select/attention take the GPU's scores /
     indices as inputs, and the end-to-end index sets are compared too)."""
-    q, k, vv, s, cu = _host(inp)
+    q, k, vv, s, cu = _host(inp, rows)
     v_dev = inp.v if v is None else v
     if v is not None:
         vv = v.detach().cpu().double().numpy()
@@ -221,3 +227,36 @@ def test_packed_workload_sampled():
     wl = workloads.PACKED
     inp, rows = _sampled(wl, 12)
     run_and_check(inp, wl.block_size, wl.topk, wl.window, rows=rows)
+
+
+@pytest.mark.slow
+def test_long_context_workload_sampled():
+    wl = workloads.LONG
+    inp, rows = _sampled(wl, 16)
+    run_and_check(inp, wl.block_size, wl.topk, wl.window, rows=rows)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("topk", [8, 16, 32, 64])
+def test_sweep_workload_sampled(topk):
+    wl = workloads.sweep(topk)
+    inp, rows = _sampled(wl, 5)
+    run_and_check(inp, wl.block_size, wl.topk, wl.window, rows=rows)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("window", [256, 1024, 4096])
+def test_sweep_swa_layer_sampled(window):
+    """The separate SWA-only layer of the sweep: Dk 192, Dv 128."""
+    wl = workloads.sweep_swa(window)
+    inp, rows = _sampled(wl, 6)
+    assert hs.path(hs.HS_OP_SWA_MQA, wl.dtype, 64, 192, 128, 64) == hs.HS_PATH_TCGEN05
+    q, k, vv, s, cu = _host(inp, rows)
+    wout, wlse = hs.hs_swa_mqa_fwd(inp.q, inp.k, inp.v, inp.cu_seqlens, inp.max_seqlen, window,
+                                   inp.sink)
+    torch.cuda.synchronize()
+    hs.poll_status()
+    rows_t = torch.as_tensor(rows, device=DEV)
+    ref = O.swa_mqa_fwd(q, k, vv, cu, window, sink=s, rows=rows)
+    P.check_out(wout[rows_t], ref["out"], "swa out")
+    P.check_lse(wlse[rows_t], ref["lse"], "swa lse")
