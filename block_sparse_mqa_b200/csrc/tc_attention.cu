@@ -556,6 +556,23 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
         const bool resc = i > 0 && sh->rescale[wg][gt & 1] != 0;
         ++gt;
+        // exp2(x - m_h) for heads hb..hb+31 of row r, packed as bf16 pairs,
+        // before waiting for the P^T buffer: after PV of the previous tile
+        // has released it only the stores remain
+        if (resc) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) lpart[k] *= sh->alpha[hb + k];
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float e0 = fast_exp2(x[2 * k] - sh->mrun[hb + 2 * k]);
+          const float e1 = fast_exp2(x[2 * k + 1] - sh->mrun[hb + 2 * k + 1]);
+          lpart[2 * k] += e0;
+          lpart[2 * k + 1] += e1;
+          __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
+          pk[k] = *reinterpret_cast<uint32_t*>(&pr);
+        }
         // P^T may be rewritten once PV of the previous tile has read it
         if (i > 0) {
           if (!mbar_wait(&sh->pvdone, npv & 1, lim)) { ok = false; break; }
@@ -576,27 +593,14 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
             tmem_st32(ta, w);
           }
           tmem_st_wait();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) lpart[k] *= sh->alpha[hb + k];
         }
-        // P^T row r, heads hb..hb+31: exp2(x - m_h) as bf16, 128-byte swizzled
+        // P^T row r, 128-byte swizzled
         uint8_t* prow = pbuf + r * 128;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int h0 = q4 * 8 + 2 * k;
-            const float e0 = fast_exp2(x[h0] - sh->mrun[hb + h0]);
-            const float e1 = fast_exp2(x[h0 + 1] - sh->mrun[hb + h0 + 1]);
-            lpart[h0] += e0;
-            lpart[h0 + 1] += e1;
-            __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
-            w4[k] = *reinterpret_cast<uint32_t*>(&pr);
-          }
           const int cidx = 4 * wg + q4;
           *reinterpret_cast<uint4*>(prow + ((cidx ^ (r & 7)) << 4)) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
@@ -623,16 +627,34 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       if (!mbar_wait(&sh->ofull, ntok & 1, lim)) { ok = false; break; }
       tc_fence_after();
       if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
-      __nv_bfloat16* orow = p.out + ((int64_t)t * kH + hb) * dvs;
-      for (int c = 0; c < p.nvc; ++c) {
-        uint32_t w[32];
-        tmem_ld32(lane_base + c * kH + hb, w);
-        tmem_ld_wait();
-        reg_fence(w);
+      // O^T chunk c (dv rows x this warpgroup's 32 heads) is normalised,
+      // staged as [head][128 dv] bf16 in this warpgroup's half of the P^T
+      // buffer (free: the token's last PV is complete) and written out as
+      // 16-byte stores, a head's 256 contiguous bytes per half-warp.  No wait
+      // inside this loop can fail, so all 128 threads meet each named barrier.
+      {
+        __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(pbuf) + wg * (32 * 128);
+        __nv_bfloat16* obase = p.out + ((int64_t)t * kH + hb) * dvs;
+        float ls[32];
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          orow[(int64_t)k * dvs + c * 128 + r] =
-              __float2bfloat16_rn(__uint_as_float(w[k]) * sh->lsum[hb + k]);
+        for (int k = 0; k < 32; ++k) ls[k] = sh->lsum[hb + k];
+        for (int c = 0; c < p.nvc; ++c) {
+          uint32_t w[32];
+          tmem_ld32(lane_base + c * kH + hb, w);
+          tmem_ld_wait();
+          reg_fence(w);
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            stage[k * 128 + r] = __float2bfloat16_rn(__uint_as_float(w[k]) * ls[k]);
+          named_bar(1 + wg, 128);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int u = r + 128 * q4;  // 16-byte unit: head u / 16, dv 8 (u % 16)
+            const uint4 v = reinterpret_cast<const uint4*>(stage)[u];
+            *reinterpret_cast<uint4*>(obase + (int64_t)(u >> 4) * dvs + c * 128 + (u & 15) * 8) = v;
+          }
+          named_bar(1 + wg, 128);
+        }
       }
       tc_fence_before();
       mbar_arrive(&sh->oempty);
@@ -661,7 +683,7 @@ bool tc_attention_supported(int num_heads, int dk, int dv, int block_size, bool 
 bool tc_attention_eligible(const AttnArgs& a) {
   const Problem& p = a.p;
   auto al16 = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; };
-  return al16(p.q) && al16(p.k) && al16(p.v) && p.q_row_stride % 8 == 0 &&
+  return al16(p.q) && al16(p.k) && al16(p.v) && al16(a.out) && p.q_row_stride % 8 == 0 &&
          p.q_head_stride % 8 == 0 && p.k_row_stride % 8 == 0 && p.v_row_stride % 8 == 0;
 }
 
