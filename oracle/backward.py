@@ -31,9 +31,10 @@ is ``dout``.  Per query token t with key set S_t, head h, s_j = scale *
     dsink_h += -p_sink * delta                (summed over t)
 
 The sink row follows from out depending on sink_h only through lse, and
-d lse / d sink_h = p_sink.  All arithmetic is float64; sums over keys and
-heads are matrix products of the library routine (numpy), sums over tokens
-run in ascending token order.
+d lse / d sink_h = p_sink.  A token with an empty key set (an idx row without
+a usable block) has out = 0, lse = sink and contributes no gradient.  All
+arithmetic is float64; sums over keys and heads are matrix products of the
+library routine (numpy), sums over tokens run in ascending token order.
 """
 
 from __future__ import annotations
@@ -58,8 +59,12 @@ def attend_bwd(q_t, keys, k, v, sink, scale: float, dout_t):
     kk = _f64(k)[keys]
     vv = _f64(v)[keys]
     do = _f64(dout_t)
-    s = scale * (q_t @ kk.T)                               # [H, n]
     sk = np.full(H, -np.inf) if sink is None else _f64(sink).reshape(H)
+    if len(keys) == 0:  # empty key set: out = 0, lse = sink, no gradient
+        z = np.zeros
+        return (z(q_t.shape), z((0, q_t.shape[1])), z((0, vv.shape[1])), z(H), z(H),
+                z((H, vv.shape[1])), sk.copy())
+    s = scale * (q_t @ kk.T)                               # [H, n]
     m = np.maximum(s.max(axis=1), sk)
     z = np.exp(s - m[:, None]).sum(axis=1) + np.exp(sk - m)
     lse = m + np.log(z)

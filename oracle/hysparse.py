@@ -275,15 +275,18 @@ def attend(q_t, keys, k, v, sink, scale: float):
         lse_nosink = log(sum_j exp(s_j))
         out[h]     = sum_j exp(s_j - lse) v[j]
 
-    ``sink`` None means no sink (equivalently -inf).  Returns
+    ``sink`` None means no sink (equivalently -inf).  An empty key set (an
+    idx row without a usable block) gives out = 0 and lse = sink.  Returns
     (out [H, Dv], lse [H], lse_nosink [H]).
     """
     q_t = _f64(q_t)
     H = q_t.shape[0]
     kk = _f64(k)[keys]
     vv = _f64(v)[keys]
-    s = scale * (q_t @ kk.T)                              # [H, n]
     sk = np.full(H, -np.inf) if sink is None else _f64(sink).reshape(H)
+    if len(keys) == 0:  # no usable block: the softmax holds only the sink
+        return np.zeros((H, vv.shape[1])), sk.copy(), np.full(H, -np.inf)
+    s = scale * (q_t @ kk.T)                              # [H, n]
     m = np.maximum(s.max(axis=1), sk)                     # finite: n >= 1
     z = np.exp(s - m[:, None]).sum(axis=1)
     zs = np.exp(sk - m)

@@ -107,6 +107,8 @@ def test_backward_matches_torch_autograd(kind, with_sink):
     if kind == "sparse":
         B, K = 4, 3
         idx = _idx(q, k, cu, B, K)
+        if with_sink:  # a row without a usable block: only the sink is left
+            idx[30] = -1
         g = OB.sparse_mqa_bwd(q, k, v, dout, idx, cu, B, sink=sink)
         mask = _mask_sparse(T, cu, idx, B)
     else:
