@@ -163,6 +163,9 @@ int hs_path(int op, hs_dtype dtype, int num_heads, int dk, int dv, int block_siz
           hs::tc_block_score_supported(num_heads, dk, block_size, 0))
         return HS_PATH_TCGEN05;
       return HS_PATH_SIMT;
+    case HS_OP_SPARSE_MQA_BWD:
+    case HS_OP_SWA_MQA_BWD:
+      return HS_PATH_SIMT;
     case HS_OP_SPARSE_MQA:
     case HS_OP_SWA_MQA:
       if (dtype == HS_BF16 && !g_force_simt.load() &&
@@ -176,6 +179,9 @@ int hs_path(int op, hs_dtype dtype, int num_heads, int dk, int dv, int block_siz
 size_t hs_workspace_size(int op, int total_tokens, int num_docs, int max_seqlen, int num_heads,
                          int dk, int dv, hs_dtype dtype, int block_size) {
   (void)dv;
+  if ((op == HS_OP_SPARSE_MQA_BWD || op == HS_OP_SWA_MQA_BWD) && total_tokens > 0 &&
+      num_heads > 0)
+    return hs::simt_backward_workspace(total_tokens, num_heads);
   if (op != HS_OP_BLOCK_SCORE || total_tokens <= 0 || !valid_block(block_size)) return 0;
   const int nbmax = nbmax_of(max_seqlen, block_size);
   if (dtype == HS_BF16 && !g_force_simt.load() &&
@@ -338,6 +344,89 @@ hs_status hs_swa_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_str
   return attention_common(a, false, q, q_row_stride, q_head_stride, k, k_row_stride, v,
                           v_row_stride, cu_seqlens, num_docs, total_tokens, max_seqlen,
                           num_heads, dk, dv, dtype, softmax_scale, sink, out, lse, stream);
+}
+
+static hs_status backward_common(hs::BwdArgs& a, bool sparse, const void* q, int64_t qrs,
+                                 int64_t qhs, const void* k, int64_t krs, const void* v,
+                                 int64_t vrs, const int32_t* cu, int num_docs, int total_tokens,
+                                 int max_seqlen, int num_heads, int dk, int dv, hs_dtype dtype,
+                                 float scale, const float* sink, const void* out,
+                                 const float* lse, const void* dout, float* dq, float* dkey,
+                                 float* dval, float* dsink, void* workspace,
+                                 size_t workspace_bytes, hs_stream_t stream) {
+  hs_status r = check_problem(a.p, q, qrs, qhs, k, krs, cu, num_docs, total_tokens, max_seqlen,
+                              num_heads, dk, dv, dtype, scale);
+  if (r != HS_OK) return r;
+  if (dv < 1) return fail(HS_ERR_UNSUPPORTED, "dv must be >= 1");
+  if (!v) return fail(HS_ERR_INVALID_ARG, "v is NULL");
+  if (vrs < dv) return fail(HS_ERR_INVALID_ARG, "v_row_stride %lld < dv", (long long)vrs);
+  if (!out || !lse || !dout) return fail(HS_ERR_INVALID_ARG, "out, lse or dout is NULL");
+  if (!dq || !dkey || !dval) return fail(HS_ERR_INVALID_ARG, "dq, dk or dv is NULL");
+  a.p.v = v;
+  a.p.v_row_stride = vrs;
+  a.sink = sink;
+  a.out = out;
+  a.lse = lse;
+  a.dout = dout;
+  a.dq = dq;
+  a.dkey = dkey;
+  a.dval = dval;
+  a.dsink = dsink;
+  if (total_tokens == 0) return HS_OK;
+  const size_t need = hs::simt_backward_workspace(total_tokens, num_heads);
+  if (!workspace || workspace_bytes < need)
+    return fail(HS_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                workspace ? workspace_bytes : (size_t)0);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 15) != 0)
+    return fail(HS_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+  a.workspace = workspace;
+  r = status_ptr(&a.p.status);
+  if (r != HS_OK) return r;
+  return launched(hs::launch_simt_backward(a, sparse, stream),
+                  sparse ? "simt sparse attention backward" : "simt swa attention backward");
+}
+
+hs_status hs_sparse_mqa_bwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                            const void* k, int64_t k_row_stride, const void* v,
+                            int64_t v_row_stride, const int32_t* cu_seqlens, int num_docs,
+                            int total_tokens, int max_seqlen, int num_heads, int dk, int dv,
+                            hs_dtype dtype, float softmax_scale, const int32_t* idx, int topk,
+                            int block_size, const float* sink, const void* out, const float* lse,
+                            const void* dout, float* dq, float* dkey, float* dval, float* dsink,
+                            void* workspace, size_t workspace_bytes, hs_stream_t stream) {
+  if (!valid_block(block_size))
+    return fail(HS_ERR_UNSUPPORTED, "block_size %d not in {16, 32, 64, 128}", block_size);
+  if (topk < 1 || topk > 256) return fail(HS_ERR_UNSUPPORTED, "topk %d not in [1, 256]", topk);
+  if (!idx) return fail(HS_ERR_INVALID_ARG, "idx is NULL");
+  hs::BwdArgs a{};
+  a.idx = idx;
+  a.topk = topk;
+  a.block_size = block_size;
+  a.window = 0;
+  return backward_common(a, true, q, q_row_stride, q_head_stride, k, k_row_stride, v,
+                         v_row_stride, cu_seqlens, num_docs, total_tokens, max_seqlen, num_heads,
+                         dk, dv, dtype, softmax_scale, sink, out, lse, dout, dq, dkey, dval,
+                         dsink, workspace, workspace_bytes, stream);
+}
+
+hs_status hs_swa_mqa_bwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                         const void* k, int64_t k_row_stride, const void* v, int64_t v_row_stride,
+                         const int32_t* cu_seqlens, int num_docs, int total_tokens,
+                         int max_seqlen, int num_heads, int dk, int dv, hs_dtype dtype,
+                         float softmax_scale, int window, const float* sink, const void* out,
+                         const float* lse, const void* dout, float* dq, float* dkey, float* dval,
+                         float* dsink, void* workspace, size_t workspace_bytes,
+                         hs_stream_t stream) {
+  if (window < 1) return fail(HS_ERR_INVALID_ARG, "window %d < 1", window);
+  hs::BwdArgs a{};
+  a.idx = nullptr;
+  a.topk = 0;
+  a.block_size = 64;
+  a.window = window;
+  return backward_common(a, false, q, q_row_stride, q_head_stride, k, k_row_stride, v,
+                         v_row_stride, cu_seqlens, num_docs, total_tokens, max_seqlen, num_heads,
+                         dk, dv, dtype, softmax_scale, sink, out, lse, dout, dq, dkey, dval,
+                         dsink, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

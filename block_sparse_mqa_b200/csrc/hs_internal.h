@@ -44,12 +44,31 @@ struct AttnArgs {
   float* lse;
 };
 
+// Backward of the attention calls (after host validation).
+struct BwdArgs {
+  Problem p;
+  const int32_t* idx;  // sparse only
+  int topk, block_size;
+  int window;          // swa only
+  const float* sink;   // may be null
+  const void* out;
+  const float* lse;
+  const void* dout;
+  float* dq;
+  float* dkey;
+  float* dval;
+  float* dsink;        // may be null
+  void* workspace;     // simt_backward_workspace() bytes
+};
+
 // Launchers; each returns cudaSuccess or the launch error.
 cudaError_t launch_simt_block_score(const ScoreArgs& a, cudaStream_t s);
 cudaError_t launch_select_topk(const float* block_score, int nb_stride, const int32_t* cu,
                                int num_docs, int total_tokens, int max_seqlen, int block_size,
                                int topk, int32_t* idx, int* status, cudaStream_t s);
 cudaError_t launch_simt_attention(const AttnArgs& a, bool sparse, cudaStream_t s);
+size_t simt_backward_workspace(int total_tokens, int num_heads);
+cudaError_t launch_simt_backward(const BwdArgs& a, bool sparse, cudaStream_t s);
 
 // Shared-memory bytes the CUDA-core block-score kernel needs (0 if it cannot run).
 size_t simt_block_score_smem(int num_heads, int dk, int nbmax);

@@ -35,6 +35,8 @@ HS_OP_BLOCK_SCORE = 0
 HS_OP_SELECT_TOPK = 1
 HS_OP_SPARSE_MQA = 2
 HS_OP_SWA_MQA = 3
+HS_OP_SPARSE_MQA_BWD = 4
+HS_OP_SWA_MQA_BWD = 5
 
 HS_PATH_SIMT = 0
 HS_PATH_TCGEN05 = 1
@@ -44,7 +46,7 @@ EXPORTS = (
     "hs_block_score", "hs_select_topk", "hs_sparse_mqa_fwd", "hs_swa_mqa_fwd",
     "hs_workspace_size", "hs_path", "hs_poll_status", "hs_set_force_simt",
     "hs_selftest_wait", "hs_status_string", "hs_last_error", "hs_version",
-    "hs_block_score_static",
+    "hs_block_score_static", "hs_sparse_mqa_bwd", "hs_swa_mqa_bwd",
 )
 
 
@@ -81,6 +83,12 @@ def lib() -> ctypes.CDLL:
                                     _vp]
     L.hs_swa_mqa_fwd.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _int, _int, _int,
                                  _int, _int, _int, _int, _flt, _int, _vp, _vp, _vp, _vp]
+    L.hs_sparse_mqa_bwd.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _int, _int, _int,
+                                    _int, _int, _int, _int, _flt, _vp, _int, _int, _vp, _vp, _vp,
+                                    _vp, _vp, _vp, _vp, _vp, _vp, _szt, _vp]
+    L.hs_swa_mqa_bwd.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _int, _int, _int,
+                                 _int, _int, _int, _int, _flt, _int, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _vp, _vp, _vp, _szt, _vp]
     L.hs_workspace_size.argtypes = [_int] * 9
     L.hs_workspace_size.restype = _szt
     L.hs_path.argtypes = [_int] * 6
@@ -94,7 +102,8 @@ def lib() -> ctypes.CDLL:
     L.hs_last_error.argtypes = []
     L.hs_last_error.restype = ctypes.c_char_p
     for fn in ("hs_block_score", "hs_select_topk", "hs_sparse_mqa_fwd", "hs_swa_mqa_fwd",
-               "hs_poll_status", "hs_block_score_static"):
+               "hs_poll_status", "hs_block_score_static", "hs_sparse_mqa_bwd",
+               "hs_swa_mqa_bwd"):
         getattr(L, fn).restype = _int
     _lib = L
     return L
@@ -279,6 +288,67 @@ def hs_swa_mqa_fwd(q, k, v, cu_seqlens, max_seqlen: int, window: int, sink=None,
         cu_seqlens.numel() - 1, T, int(max_seqlen), H, Dk, v.shape[1], _dtype_code(q),
         float(softmax_scale), int(window), _ptr(sink), _ptr(o), _ptr(l), _stream(q.device)))
     return o, l
+
+
+def _bwd_prep(q, k, v, out, lse, dout, cu_seqlens, sink, op, max_seqlen, grads, workspace):
+    _need_cuda(q, k, v, out, lse, dout, cu_seqlens, sink)
+    qrs, qhs, krs = _qk_strides(q, k)
+    if v.dim() != 2 or v.stride(1) != 1:
+        raise ValueError("v must be [T, Dv] with contiguous rows")
+    for name, t in (("out", out), ("lse", lse), ("dout", dout)):
+        if not t.is_contiguous():
+            raise ValueError("%s must be contiguous" % name)
+    if lse.dtype != torch.float32 or out.dtype != q.dtype or dout.dtype != q.dtype:
+        raise ValueError("lse must be float32; out and dout in q's dtype")
+    T, H, Dk = q.shape
+    Dv = v.shape[1]
+    dev = q.device
+    f32 = torch.float32
+    if grads is None:
+        grads = (torch.empty((T, H, Dk), device=dev, dtype=f32),
+                 torch.empty((T, Dk), device=dev, dtype=f32),
+                 torch.empty((T, Dv), device=dev, dtype=f32),
+                 torch.empty((H,), device=dev, dtype=f32) if sink is not None else None)
+    for g in grads:
+        if g is not None and (g.dtype != f32 or not g.is_contiguous()):
+            raise ValueError("gradient outputs must be contiguous float32")
+    need = workspace_size(op, T, cu_seqlens.numel() - 1, max_seqlen, H, Dk, Dv, q.dtype, 64)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    return qrs, qhs, krs, grads, workspace
+
+
+def hs_sparse_mqa_bwd(q, k, v, idx, cu_seqlens, max_seqlen: int, block_size: int, out, lse,
+                      dout, sink=None, softmax_scale: float = 0.0, grads=None, workspace=None):
+    """Backward of step 3.  Returns (dq [T,H,Dk], dk [T,Dk], dv [T,Dv],
+    dsink [H] or None), all float32."""
+    if idx.dtype != torch.int32 or not idx.is_contiguous():
+        raise ValueError("idx must be contiguous int32 [T, topk]")
+    qrs, qhs, krs, g, ws = _bwd_prep(q, k, v, out, lse, dout, cu_seqlens, sink,
+                                     HS_OP_SPARSE_MQA_BWD, max_seqlen, grads, workspace)
+    T, H, Dk = q.shape
+    _check(lib().hs_sparse_mqa_bwd(
+        _ptr(q), qrs, qhs, _ptr(k), krs, _ptr(v), v.stride(0), _ptr(cu_seqlens),
+        cu_seqlens.numel() - 1, T, int(max_seqlen), H, Dk, v.shape[1], _dtype_code(q),
+        float(softmax_scale), _ptr(idx), idx.shape[1], int(block_size), _ptr(sink), _ptr(out),
+        _ptr(lse), _ptr(dout), _ptr(g[0]), _ptr(g[1]), _ptr(g[2]), _ptr(g[3]), _ptr(ws),
+        0 if ws is None else ws.numel(), _stream(q.device)))
+    return g
+
+
+def hs_swa_mqa_bwd(q, k, v, cu_seqlens, max_seqlen: int, window: int, out, lse, dout,
+                   sink=None, softmax_scale: float = 0.0, grads=None, workspace=None):
+    """Backward of step 4.  Returns (dq, dk, dv, dsink or None), float32."""
+    qrs, qhs, krs, g, ws = _bwd_prep(q, k, v, out, lse, dout, cu_seqlens, sink,
+                                     HS_OP_SWA_MQA_BWD, max_seqlen, grads, workspace)
+    T, H, Dk = q.shape
+    _check(lib().hs_swa_mqa_bwd(
+        _ptr(q), qrs, qhs, _ptr(k), krs, _ptr(v), v.stride(0), _ptr(cu_seqlens),
+        cu_seqlens.numel() - 1, T, int(max_seqlen), H, Dk, v.shape[1], _dtype_code(q),
+        float(softmax_scale), int(window), _ptr(sink), _ptr(out), _ptr(lse), _ptr(dout),
+        _ptr(g[0]), _ptr(g[1]), _ptr(g[2]), _ptr(g[3]), _ptr(ws),
+        0 if ws is None else ws.numel(), _stream(q.device)))
+    return g
 
 
 def hs_forward(q, k, v, cu_seqlens, max_seqlen: int, block_size: int, topk: int, window: int,

@@ -1,5 +1,5 @@
 /*
- * hs.h -- C ABI of libhs, the B200 (sm_100a) HySparse MQA forward path.
+ * hs.h -- C ABI of libhs, the B200 (sm_100a) HySparse MQA attention path.
  *
  * The method: "HySparse MQA sparse attention (FA4 block scoring + SWA MQA +
  * block-sparse DSA gather)", PaddleFleet pull request 1470 ("Core" list and
@@ -13,6 +13,10 @@
  *   hs_select_topk     per-query top-k key blocks inside its document
  *   hs_sparse_mqa_fwd  softmax attention over the selected blocks + sink
  *   hs_swa_mqa_fwd     sliding-window attention + sink (Dk != Dv allowed)
+ *
+ * and two calls give the backward of the two attention steps:
+ *   hs_sparse_mqa_bwd  dq, dk, dv and the sink gradient of hs_sparse_mqa_fwd
+ *   hs_swa_mqa_bwd     the same for hs_swa_mqa_fwd
  *
  * Conventions shared by every call
  * --------------------------------
@@ -88,7 +92,9 @@ typedef enum hs_op {
   HS_OP_BLOCK_SCORE = 0,
   HS_OP_SELECT_TOPK = 1,
   HS_OP_SPARSE_MQA = 2,
-  HS_OP_SWA_MQA = 3
+  HS_OP_SWA_MQA = 3,
+  HS_OP_SPARSE_MQA_BWD = 4,
+  HS_OP_SWA_MQA_BWD = 5
 } hs_op;
 
 /* Kernel family a call will use, as returned by hs_path(). */
@@ -201,6 +207,72 @@ hs_status hs_swa_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_str
                          void* out, float* lse, hs_stream_t stream);
 
 /*
+ * Backward of step 3 (block-sparse MQA with a per-head sink).
+ * Source: pull request 1470, "Core" list (the block-sparse MQA and SWA
+ * kernels come with backward passes; the learnable per-head attn_sink has an
+ * analytic gradient) and per-file table (block-sparse DSA gather backend:
+ * analytic sink gradient).  The pages give no formulas; this is the exact
+ * gradient of hs_sparse_mqa_fwd for a loss L with dL/dout = dout.  With the
+ * forward's key sets S_t, s_j = scale * <q[t,h], k[j]>, p_j = exp(s_j -
+ * lse[t,h]) (lse includes the sink) and delta[t,h] = <dout[t,h], out[t,h]>:
+ *   ds_j     = p_j * (<dout[t,h], v[j]> - delta[t,h])
+ *   dq[t,h]  = scale * sum_{j in S_t} ds_j * k[j]
+ *   dk[j]    = scale * sum over (t,h) with j in S_t of ds_j * q[t,h]
+ *   dv[j]    = sum over (t,h) with j in S_t of p_j * dout[t,h]
+ *   dsink[h] = -sum_t exp(sink[h] - lse[t,h]) * delta[t,h]
+ *
+ * Inputs are those of the forward call plus:
+ *   out, dout  [T, H, Dv] of `dtype`, contiguous: the forward's output and
+ *              the gradient of the loss with respect to it.
+ *   lse        [T, H] fp32: the forward's lse (sink included).
+ * Outputs (fp32, contiguous, fully overwritten; keys no query selected get
+ * zero gradients):
+ *   dq         [T, H, Dk]
+ *   dkey       [T, Dk]   gradient with respect to the T rows of k
+ *   dval       [T, Dv]   gradient with respect to the T rows of v (when v
+ *                        aliases the first Dv columns of k, the caller adds
+ *                        dval into those columns of dkey)
+ *   dsink      [H], or NULL to skip; ignored when sink is NULL.
+ *   workspace  device scratch of at least hs_workspace_size(
+ *              HS_OP_SPARSE_MQA_BWD, ...) bytes (8 * T * H), 16-byte
+ *              aligned; its contents on entry do not matter; concurrent
+ *              calls must not share one.  A missing or short workspace is
+ *              HS_ERR_WORKSPACE before any device work.
+ * idx entries follow the forward's rule; offending entries are skipped and
+ * reported as HS_ERR_INVALID_INDEX.  Results are deterministic (every sum
+ * runs in a fixed order).
+ */
+hs_status hs_sparse_mqa_bwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                            const void* k, int64_t k_row_stride,
+                            const void* v, int64_t v_row_stride,
+                            const int32_t* cu_seqlens, int num_docs, int total_tokens,
+                            int max_seqlen, int num_heads, int dk, int dv, hs_dtype dtype,
+                            float softmax_scale, const int32_t* idx, int topk,
+                            int block_size, const float* sink,
+                            const void* out, const float* lse, const void* dout,
+                            float* dq, float* dkey, float* dval, float* dsink,
+                            void* workspace, size_t workspace_bytes, hs_stream_t stream);
+
+/*
+ * Backward of step 4 (sliding-window MQA with a per-head sink).
+ * Source: pull request 1470, "Core" list (SWA sliding-window MQA) and
+ * per-file table (windowed_mqa_attn*.py: fwd/bwd with Dk != Dv, attn_sink and
+ * a guard for ragged sequence lengths in the backward).  Same formulas,
+ * arguments and outputs as hs_sparse_mqa_bwd with the forward's window key
+ * sets j in [max(bos, t - window + 1), t]; workspace size from
+ * hs_workspace_size(HS_OP_SWA_MQA_BWD, ...).
+ */
+hs_status hs_swa_mqa_bwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                         const void* k, int64_t k_row_stride,
+                         const void* v, int64_t v_row_stride,
+                         const int32_t* cu_seqlens, int num_docs, int total_tokens,
+                         int max_seqlen, int num_heads, int dk, int dv, hs_dtype dtype,
+                         float softmax_scale, int window, const float* sink,
+                         const void* out, const float* lse, const void* dout,
+                         float* dq, float* dkey, float* dval, float* dsink,
+                         void* workspace, size_t workspace_bytes, hs_stream_t stream);
+
+/*
  * Step 1 for callers that cannot allocate device memory.
  * The method has no counterpart of this call; it is a deployment aid.
  *
@@ -237,8 +309,8 @@ hs_status hs_block_score_static(const void* q, int64_t q_row_stride, int64_t q_h
 
 /* ---------------------------------------------------------------- helpers */
 
-/* Bytes of `workspace` that op needs for these sizes (0 = none).  Only
- * HS_OP_BLOCK_SCORE uses a workspace. */
+/* Bytes of `workspace` that op needs for these sizes (0 = none).
+ * HS_OP_BLOCK_SCORE and the two backward ops use a workspace. */
 size_t hs_workspace_size(int op, int total_tokens, int num_docs, int max_seqlen,
                          int num_heads, int dk, int dv, hs_dtype dtype, int block_size);
 

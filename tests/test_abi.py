@@ -109,6 +109,40 @@ def test_attention_rejects_bad_arguments():
     assert L.hs_swa_mqa_fwd(*no_dv, 16, None, p, p, None) == hs.HS_ERR_UNSUPPORTED
 
 
+
+def test_backward_rejects_bad_arguments():
+    L = hs.lib()
+    p = ctypes.c_void_p(1)
+    ws = ctypes.c_void_p(256)  # 16-byte aligned stand-in
+    T, H = 100, 64
+    need = L.hs_workspace_size(hs.HS_OP_SPARSE_MQA_BWD, T, 1, 100, H, 576, 512, hs.HS_BF16, 64)
+    assert need == 8 * T * H
+    assert L.hs_workspace_size(hs.HS_OP_SWA_MQA_BWD, T, 1, 100, H, 576, 512, hs.HS_BF16, 64) == need
+    assert L.hs_path(hs.HS_OP_SPARSE_MQA_BWD, hs.HS_BF16, H, 576, 512, 64) == hs.HS_PATH_SIMT
+    args = [p, 64 * 576, 576, p, 576, p, 512, p, 1, T, 100, H, 576, 512, hs.HS_BF16, 0.0]
+    tail = [p, p, p, p, p, p, None]  # out, lse, dout, dq, dk, dv, dsink
+    # sparse: bad topk / idx / block, missing gradient outputs, workspace
+    assert L.hs_sparse_mqa_bwd(*args, p, 0, 64, None, *tail, ws, need, None) == hs.HS_ERR_UNSUPPORTED
+    assert L.hs_sparse_mqa_bwd(*args, None, 4, 64, None, *tail, ws, need, None) == hs.HS_ERR_INVALID_ARG
+    assert L.hs_sparse_mqa_bwd(*args, p, 4, 8, None, *tail, ws, need, None) == hs.HS_ERR_UNSUPPORTED
+    no_dq = list(tail)
+    no_dq[3] = None
+    assert L.hs_sparse_mqa_bwd(*args, p, 4, 64, None, *no_dq, ws, need, None) == hs.HS_ERR_INVALID_ARG
+    no_dout = list(tail)
+    no_dout[2] = None
+    assert L.hs_sparse_mqa_bwd(*args, p, 4, 64, None, *no_dout, ws, need, None) == hs.HS_ERR_INVALID_ARG
+    assert L.hs_sparse_mqa_bwd(*args, p, 4, 64, None, *tail, None, need, None) == hs.HS_ERR_WORKSPACE
+    assert L.hs_sparse_mqa_bwd(*args, p, 4, 64, None, *tail, ws, need - 1, None) == hs.HS_ERR_WORKSPACE
+    odd = ctypes.c_void_p(258)
+    assert L.hs_sparse_mqa_bwd(*args, p, 4, 64, None, *tail, odd, need, None) == hs.HS_ERR_INVALID_ARG
+    # swa: window 0, short workspace
+    assert L.hs_swa_mqa_bwd(*args, 0, None, *tail, ws, need, None) == hs.HS_ERR_INVALID_ARG
+    assert L.hs_swa_mqa_bwd(*args, 16, None, *tail, ws, 0, None) == hs.HS_ERR_WORKSPACE
+    # no tokens: nothing to do, no workspace needed
+    empty = list(args)
+    empty[9] = 0
+    assert L.hs_swa_mqa_bwd(*empty, 16, None, *tail, None, 0, None) == hs.HS_OK
+
 def test_binding_refuses_cpu_tensors():
     import torch
     q = torch.zeros(4, 2, 8)
