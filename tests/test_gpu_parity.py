@@ -40,9 +40,10 @@ def _expect_path(op, inp, B):
 
 
 def run_and_check(inp, B, K, W, rows=None, sink=True, scale=0.0, v=None, check_paths=None):
-    """Run the four steps on the GPU and compare each against the oracle
-    (stage-isolated: the oracle's select/attention take the GPU's scores /
-    indices as inputs, and the end-to-end index sets are compared too)."""
+    """Run the four steps on the GPU and compare each against the oracle.
+    Stages are isolated without feeding GPU results to the oracle: the GPU
+    re-runs selection on the oracle's scores and sparse attention on the
+    oracle's index sets; the end-to-end index sets are compared too."""
     q, k, vv, s, cu = _host(inp, rows)
     v_dev = inp.v if v is None else v
     if v is not None:
@@ -70,17 +71,33 @@ def run_and_check(inp, B, K, W, rows=None, sink=True, scale=0.0, v=None, check_p
     P.check_scores(bs[rows_t], ref1["block_score"])
     if blse is not None:
         P.check_lse(blse[rows_t][:, :, :nb], ref1["block_lse"], "block_lse")
-    # select: bit-exact on the GPU's own scores, near-tie rule against the oracle's
-    bs_rows = bs[rows_t].double().cpu().numpy()
+    # select, bit-exact: the GPU selects on the oracle's scores rounded to
+    # fp32 on the host (rows outside the sample hold zeros and are ignored),
+    # and the oracle selects on the same fp32 values
+    nbs = bs.shape[1]
+    bs32 = np.zeros((len(rr), nbs), dtype=np.float32)
+    bs32[:, :nb] = ref1["block_score"].astype(np.float32)
+    bs_in = torch.zeros((T, nbs), device=DEV, dtype=torch.float32)
+    bs_in[rows_t] = torch.as_tensor(bs32, device=DEV)
+    idx_on_ref = hs.hs_select_topk(bs_in, inp.cu_seqlens, inp.max_seqlen, B, K)
+    ref_idx32 = O.select_topk(bs32[:, :nb].astype(np.float64), cu, B, K, rows=rr, total_tokens=T)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(idx_on_ref[rows_t].cpu().numpy(), ref_idx32)
+    # the end-to-end GPU index sets against the oracle's (near-tie rule)
     idx_rows = idx[rows_t].cpu().numpy()
-    ref_idx_same = O.select_topk(bs_rows, cu, B, K, rows=rr, total_tokens=T)
-    np.testing.assert_array_equal(idx_rows, ref_idx_same)
     ref_idx = O.select_topk(ref1["block_score"], cu, B, K, rows=rr, total_tokens=T)
     P.check_topk(idx_rows, ref_idx, ref1["block_score"], P.bq_rows(cu, rr, B), K)
-    # attention on the GPU's indices
-    ref3 = O.sparse_mqa_fwd(q, k, vv, idx_rows, cu, B, sink=sink_np, scale=sc, rows=rr)
-    P.check_out(out[rows_t], ref3["out"], "sparse out")
-    P.check_lse(lse[rows_t], ref3["lse"], "sparse lse")
+    # sparse attention on the oracle's index sets (uploaded for the sampled
+    # rows; the other rows keep the GPU's own, their outputs are ignored)
+    idx_mix = idx.clone()
+    idx_mix[rows_t] = torch.as_tensor(np.ascontiguousarray(ref_idx, dtype=np.int32), device=DEV)
+    out_r, lse_r = hs.hs_sparse_mqa_fwd(inp.q, inp.k, v_dev, idx_mix, inp.cu_seqlens,
+                                        inp.max_seqlen, B, sink_dev, scale)
+    torch.cuda.synchronize()
+    hs.poll_status()
+    ref3 = O.sparse_mqa_fwd(q, k, vv, ref_idx, cu, B, sink=sink_np, scale=sc, rows=rr)
+    P.check_out(out_r[rows_t], ref3["out"], "sparse out")
+    P.check_lse(lse_r[rows_t], ref3["lse"], "sparse lse")
     ref4 = O.swa_mqa_fwd(q, k, vv, cu, W, sink=sink_np, scale=sc, rows=rr)
     P.check_out(wout[rows_t], ref4["out"], "swa out")
     P.check_lse(wlse[rows_t], ref4["lse"], "swa lse")
