@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--workload", default=workloads.MAIN.name)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the (separately timed) backward of the two attention steps")
     ap.add_argument("--cpu-rows", type=int, default=1536,
                     help="query rows of the oracle sample (cpu_baseline / reference arm)")
     return ap.parse_args()
@@ -386,6 +388,9 @@ def run_ours(args, wl, world, rank):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(inp, wl, step, max(3, min(args.steps, 10)), world)
+    bwd = None
+    if not args.no_backward:
+        bwd = run_backward(inp, wl, step, cu, pk)
 
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -404,7 +409,52 @@ def run_ours(args, wl, world, rank):
         "gpu_launches": 4 * args.steps,
         "clocks": clk,
         "e2e": e2e,
+        "backward": bwd,
     }
+    return res
+
+
+def run_backward(inp, wl, step, cu, pk, reps=2):
+    """Backward of the two attention steps on the same inputs (not part of the
+    headline step): CUDA-event time per call, one untimed call first.
+    Algorithmic work per valid (query, key) pair and head: recomputed scores
+    (2 Dk), dp (2 Dv), dq (2 Dk), dk (2 Dk), dv (2 Dv) flops."""
+    T, H = wl.total_tokens, wl.num_heads
+    g = torch.Generator(device=inp.q.device)
+    g.manual_seed(123)
+    dout = torch.randn((T, H, wl.dv), generator=g, device=inp.q.device).to(wl.dtype)
+    ws = torch.empty(hs.workspace_size(hs.HS_OP_SPARSE_MQA_BWD, T, len(wl.docs()), inp.max_seqlen,
+                                       H, wl.dk, wl.dv, wl.dtype, wl.block_size),
+                     device=inp.q.device, dtype=torch.uint8)
+    calls = {
+        "sparse": lambda: hs.hs_sparse_mqa_bwd(inp.q, inp.k, inp.v, step.idx, inp.cu_seqlens,
+                                               inp.max_seqlen, wl.block_size, step.out, step.lse,
+                                               dout, inp.sink, workspace=ws),
+        "swa": lambda: hs.hs_swa_mqa_bwd(inp.q, inp.k, inp.v, inp.cu_seqlens, inp.max_seqlen,
+                                         wl.window, step.wout, step.wlse, dout, inp.sink,
+                                         workspace=ws),
+    }
+    pairs = {"sparse": sparse_pairs(step.idx, cu, wl.block_size),
+             "swa": window_pairs(wl.docs(), wl.window)}
+    res = {}
+    for name, fn in calls.items():
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = statistics.mean(ts)
+        fl = 2.0 * H * (3 * wl.dk + 2 * wl.dv) * pairs[name]
+        tf = fl / (ms / 1e3) / 1e12
+        res[name] = {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / pk["bf16_tflops"],
+                     "algorithmic_flops": fl, "path": "simt", "calls_timed": reps}
+    hs.poll_status(inp.q.device)
     return res
 
 

@@ -12,6 +12,8 @@ Modules
 -------
 hysparse
     Vectorised NumPy float64 implementation of the four steps.
+backward
+    The gradient of the two attention steps (dq, dk, dv, sink gradient).
 loops
     Pure-Python loop restatements, for brute-force checks on tiny inputs.
 
