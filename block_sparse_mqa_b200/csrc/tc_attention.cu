@@ -66,7 +66,8 @@ struct AttnParams {
   int num_docs, T, max_seqlen;
   const int32_t* idx;
   int topk, B, window;
-  int nck, nvc;  // 64-column K chunks, 128-row V chunks
+  int nck, nvc;  // 64-column K chunks, 128-row V chunks (the last may be half past Dv)
+  int dv;
   float scale_log2;
   const float* sink;
   __nv_bfloat16* out;
@@ -478,7 +479,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
     const int hb = 32 * wg;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * g4) << 16);
     const float sl2 = p.scale_log2;
-    const int dvs = p.nvc * 128;
+    const int dvs = p.dv;  // row stride of out
     uint32_t sidx = 0, npv = 0, rvph = 0, ntok = 0, gt = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.T && ok && !aborted(sh); t += G) {
@@ -651,7 +652,9 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           for (int q4 = 0; q4 < 4; ++q4) {
             const int u = r + 128 * q4;  // 16-byte unit: head u / 16, dv 8 (u % 16)
             const uint4 v = reinterpret_cast<const uint4*>(stage)[u];
-            *reinterpret_cast<uint4*>(obase + (int64_t)(u >> 4) * dvs + c * 128 + (u & 15) * 8) = v;
+            const int col = c * 128 + (u & 15) * 8;
+            if (col < dvs)  // a last chunk half past Dv holds zero rows
+              *reinterpret_cast<uint4*>(obase + (int64_t)(u >> 4) * dvs + col) = v;
           }
           named_bar(1 + wg, 128);
         }
@@ -676,7 +679,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
 bool tc_attention_supported(int num_heads, int dk, int dv, int block_size, bool sparse) {
   (void)sparse;
   return num_heads == kH && dk % 64 == 0 && dk >= 64 && dk <= 64 * kMaxQChunks &&
-         dv % 128 == 0 && dv >= 128 && dv <= 512 &&
+         dv % 64 == 0 && dv >= 64 && dv <= 512 &&
          (block_size == 16 || block_size == 32 || block_size == 64 || block_size == 128);
 }
 
@@ -720,7 +723,8 @@ cudaError_t launch_tc_attention(const AttnArgs& a, bool sparse, long long wait_l
   ap.B = a.block_size;
   ap.window = a.window;
   ap.nck = p.dk / 64;
-  ap.nvc = p.dv / 128;
+  ap.nvc = (p.dv + 127) / 128;  // a panel past Dv is zero-filled by TMA
+  ap.dv = p.dv;
   ap.scale_log2 = p.scale * kLog2e;
   ap.sink = a.sink;
   ap.out = static_cast<__nv_bfloat16*>(a.out);

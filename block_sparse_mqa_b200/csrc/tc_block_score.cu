@@ -140,15 +140,16 @@ __device__ __forceinline__ float transpose_reduce_sum(float (&v)[32]) {
   return v[0];
 }
 
-// One ring stage = three 64-column K chunks = 12 MMAs (M=128, N=128, K=16)
-// into S accumulator d.  FIRST: the stage opens the S tile (its first MMA
+// One ring stage = NC (three, fewer in the last stage when Dk is not a
+// multiple of 192) 64-column K chunks = 4 NC MMAs (M=128, N=128, K=16) into S
+// accumulator d.  FIRST: the stage opens the S tile (its first MMA
 // overwrites d).  SS_FIRST: its first chunk is the shared-memory q chunk
 // (descriptor qd), the others come from TMEM q chunks tpos, tpos+1, ...
-template <bool FIRST, bool SS_FIRST>
+template <bool FIRST, bool SS_FIRST, int NC = kChunksPerStage>
 __device__ __forceinline__ void issue_stage(uint32_t d, uint32_t tmem, int tpos, uint64_t qd,
                                             uint64_t b0, uint32_t idesc) {
 #pragma unroll
-  for (int c = 0; c < kChunksPerStage; ++c) {
+  for (int c = 0; c < NC; ++c) {
     const uint64_t bc = b0 + (uint64_t)((c * kChunkBytes) >> 4);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -268,15 +269,16 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
         // per key tile, ring stages of three K chunks in the MMA's order: the
         // shared-memory (RoPE) chunks first, then the TMEM chunks 0, 1, ...
         const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
-        const int spt = p.nck / kChunksPerStage;  // stages per key tile
+        const int spt = (p.nck + kChunksPerStage - 1) / kChunksPerStage;  // stages per key tile
         for (int kt = 0; kt < nkt && !aborted(sh); ++kt) {
           for (int st = 0; st < spt; ++st) {
+            const int nst = min(kChunksPerStage, p.nck - st * kChunksPerStage);
             if (!mbar_wait(&sh->kempty[kst], kph ^ 1, lim)) {
               give_up(sh, p.status);
               break;
             }
-            mbar_expect_tx(&sh->kfull[kst], kStageBytes);
-            for (int j = 0; j < kChunksPerStage; ++j) {
+            mbar_expect_tx(&sh->kfull[kst], nst * kChunkBytes);
+            for (int j = 0; j < nst; ++j) {
               const int pos = st * kChunksPerStage + j;
               const int ch = pos < p.nq_smem ? p.nq_tmem + pos : pos - p.nq_smem;
               tma_load_2d(stages + kst * kStageBytes + j * kChunkBytes, &kmap, &sh->kfull[kst],
@@ -339,7 +341,7 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
             kph ^= 1;
           }
         }
-        const int spt = p.nck / kChunksPerStage;
+        const int spt = (p.nck + kChunksPerStage - 1) / kChunksPerStage;
         for (int kt = 0; kt < nkt && ok; ++kt) {
           const uint32_t buf = sidx & 1, use = sidx >> 1;
           if (!mbar_wait_spin(&sh->sempty[buf], (use & 1) ^ 1, lim)) {
@@ -358,12 +360,21 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
             // tcgen05.mma costs about half the issue rate); one stage pattern
             // is chosen per stage
             const int tpos = st * kChunksPerStage - p.nq_smem;  // first TMEM chunk
+            // a shorter last stage (Dk not a multiple of 192) only occurs
+            // without a shared-memory q chunk (that needs 9 chunks)
+            const int nst = min(kChunksPerStage, p.nck - st * kChunksPerStage);
             if (st == 0 && p.nq_smem > 0)
               issue_stage<true, true>(d, tmem, tpos, qhi_desc[0], b0, idesc);
-            else if (st == 0)
-              issue_stage<true, false>(d, tmem, tpos, 0, b0, idesc);
-            else
-              issue_stage<false, false>(d, tmem, tpos, 0, b0, idesc);
+            else if (nst == kChunksPerStage) {
+              if (st == 0) issue_stage<true, false>(d, tmem, tpos, 0, b0, idesc);
+              else issue_stage<false, false>(d, tmem, tpos, 0, b0, idesc);
+            } else if (nst == 2) {
+              if (st == 0) issue_stage<true, false, 2>(d, tmem, tpos, 0, b0, idesc);
+              else issue_stage<false, false, 2>(d, tmem, tpos, 0, b0, idesc);
+            } else {
+              if (st == 0) issue_stage<true, false, 1>(d, tmem, tpos, 0, b0, idesc);
+              else issue_stage<false, false, 1>(d, tmem, tpos, 0, b0, idesc);
+            }
             issued = true;
             umma_commit(&sh->kempty[kst]);
             if (++kst == kStages) {
@@ -587,9 +598,9 @@ int grid_for(int total_tokens, int num_docs, int num_heads) {
 
 bool tc_block_score_supported(int num_heads, int dk, int block_size, int nbmax) {
   (void)nbmax;
-  // whole stages of three 64-column chunks: Dk in {192, 384, 576}
-  return (num_heads == 32 || num_heads == 64 || num_heads == 128) && dk % 192 == 0 &&
-         dk >= 192 && dk <= 64 * (kMaxTmemQ + kMaxQhi) &&
+  // 64-column chunks, at most kMaxTmemQ in TMEM and kMaxQhi in shared memory
+  return (num_heads == 32 || num_heads == 64 || num_heads == 128) && dk % 64 == 0 &&
+         dk >= 64 && dk <= 64 * (kMaxTmemQ + kMaxQhi) &&
          (block_size == 16 || block_size == 32 || block_size == 64 || block_size == 128);
 }
 

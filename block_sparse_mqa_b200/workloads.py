@@ -68,6 +68,14 @@ def sweep_swa(window: int) -> Workload:
                     doc_lengths=(32768,) * 4)
 
 
-ALL = {w.name: w for w in [TINY, MAIN, PACKED, LONG]
+# shape variants of the main workload: no RoPE chunk (Dk = 512) and a latent
+# narrower than 512 (Dv = 448), the two widths the FlashMLA constraints and
+# the value-padding note name
+NOROPE = Workload("mla_T4096_H64_dk512_dv512_bf16_B64_k16_w512", 4096, 64, 512, 512,
+                  torch.bfloat16, 64, 16, 512)
+NARROW_V = Workload("mla_T4096_H64_dk576_dv448_bf16_B64_k16_w512", 4096, 64, 576, 448,
+                    torch.bfloat16, 64, 16, 512)
+
+ALL = {w.name: w for w in [TINY, MAIN, PACKED, LONG, NOROPE, NARROW_V]
        + [sweep(k) for k in (8, 16, 32, 64)]
        + [sweep_swa(w) for w in (256, 1024, 4096)]}

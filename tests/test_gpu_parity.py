@@ -181,6 +181,20 @@ def test_other_head_counts_and_dims():
         run_and_check(inp, 16, 4, 33)
 
 
+
+@pytest.mark.parametrize("dk,dv", [(512, 512), (576, 448), (448, 256), (256, 192), (128, 64),
+                                   (64, 128)])
+def test_shape_variants_on_tensor_cores(dk, dv):
+    """Dk = 512 (no RoPE chunk, "FlashMLA sparse kernel constraints": d_qk in
+    {512, 576}), Dv below 512 natively (kv_lora_rank < 512) and other widths
+    that are multiples of 64: both block scoring and attention stay on the
+    tensor-core path."""
+    docs = [260, 71, 130]
+    inp = _gpu_inputs(sum(docs), 64, dk, dv, torch.bfloat16, docs, seed=14)
+    for op in (hs.HS_OP_BLOCK_SCORE, hs.HS_OP_SPARSE_MQA, hs.HS_OP_SWA_MQA):
+        assert _expect_path(op, inp, 64) == hs.HS_PATH_TCGEN05, (op, dk, dv)
+    run_and_check(inp, 64, 4, 100)
+
 def test_force_simt_agrees_with_default_path():
     docs = [333, 80]
     inp = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=7)
@@ -236,6 +250,14 @@ def _sampled(wl, per_doc, seed=0):
 def test_main_workload_sampled():
     wl = workloads.MAIN
     inp, rows = _sampled(wl, 48)
+    run_and_check(inp, wl.block_size, wl.topk, wl.window, rows=rows)
+
+
+@pytest.mark.parametrize("wl", [workloads.NOROPE, workloads.NARROW_V], ids=lambda w: w.name)
+def test_shape_variant_workloads_sampled(wl):
+    inp, rows = _sampled(wl, 24)
+    for op in (hs.HS_OP_BLOCK_SCORE, hs.HS_OP_SPARSE_MQA, hs.HS_OP_SWA_MQA):
+        assert _expect_path(op, inp, wl.block_size) == hs.HS_PATH_TCGEN05
     run_and_check(inp, wl.block_size, wl.topk, wl.window, rows=rows)
 
 
