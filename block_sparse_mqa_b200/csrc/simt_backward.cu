@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(const BwdParams a, i
 constexpr size_t kMaxSmem = 227 * 1024;
 
 template <typename T, bool kSparse>
-cudaError_t launch_typed(BwdParams a, cudaStream_t s) {
+cudaError_t launch_typed(BwdParams a, bool dkdv, cudaStream_t s) {
   const Problem& P = a.p;
   const int NT = P.total_tokens, H = P.num_heads;
   const int pairs = NT * H;
@@ -423,8 +423,9 @@ cudaError_t launch_typed(BwdParams a, cudaStream_t s) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  // dk, dv: key tiles of at most kKeyTile keys
-  {
+  // dk, dv: key tiles of at most kKeyTile keys (unless the caller runs the
+  // tensor-core key-major pass instead)
+  if (dkdv) {
     int G = 16, KT = kKeyTile;
     const size_t ints = 2 * kThreads * sizeof(int);
     while (KT > 4 && dkdv_smem_floats(G, KT, P.dk, P.dv) * 4 + ints > kMaxSmem) KT >>= 1;
@@ -464,9 +465,14 @@ cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, cudaStream_t s) 
   a.dsink = b.dsink;
   a.delta = static_cast<float*>(b.workspace);
   a.dsink_part = a.delta + (size_t)b.p.total_tokens * b.p.num_heads;
-  if (b.p.dtype == HS_BF16)
-    return sparse ? launch_typed<__nv_bfloat16, true>(a, s) : launch_typed<__nv_bfloat16, false>(a, s);
-  return sparse ? launch_typed<float, true>(a, s) : launch_typed<float, false>(a, s);
+  if (b.p.dtype == HS_BF16) {
+    const bool mma = mma_backward_supported(b.p);
+    cudaError_t e = sparse ? launch_typed<__nv_bfloat16, true>(a, !mma, s)
+                           : launch_typed<__nv_bfloat16, false>(a, !mma, s);
+    if (e != cudaSuccess || !mma) return e;
+    return launch_mma_dkdv(b, sparse, a.delta, s);
+  }
+  return sparse ? launch_typed<float, true>(a, true, s) : launch_typed<float, false>(a, true, s);
 }
 
 }  // namespace hs

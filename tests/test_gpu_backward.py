@@ -107,6 +107,17 @@ def test_backward_block_and_window_variants(B, K, W):
         run_backward(docs, 8, 128, 64, torch.bfloat16, kind, B=B, K=K, W=W, seed=2)
 
 
+@pytest.mark.parametrize("B,K,W,dk,dv", [(16, 3, 1, 128, 64), (32, 2, 700, 192, 128),
+                                         (128, 5, 129, 512, 448), (64, 4, 64, 64, 512)])
+def test_backward_tensor_core_variants(B, K, W, dk, dv):
+    """64 heads in bf16 take the tensor-core key-major dk/dv pass: block sizes
+    whose blocks a 32-key tile can straddle (three at B = 16), documents that
+    start off the tile grid, and Dk / Dv multiples of 64."""
+    docs = [300, 37, 180]
+    for kind in ("sparse", "swa"):
+        run_backward(docs, 64, dk, dv, torch.bfloat16, kind, B=B, K=K, W=W, seed=3)
+
+
 def test_backward_other_dims():
     # Dk != Dv, not multiples of 64; several head groups with a partial last one
     run_backward([120, 88], 20, 80, 48, torch.float32, "sparse", B=16, K=3, seed=4)
