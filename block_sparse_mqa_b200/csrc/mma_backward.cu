@@ -1,6 +1,6 @@
-// Key-major dk / dv pass of the attention backward on warp-level tensor-core
-// MMAs (mma.sync m16n8k16, bf16 in, fp32 accumulate), for bf16 inputs with
-// 64 heads, Dk and Dv multiples of 64 (Dk <= 576, Dv <= 512).
+// The dq and dk / dv passes of the attention backward on warp-level
+// tensor-core MMAs (mma.sync m16n8k16, bf16 in, fp32 accumulate), for bf16
+// inputs with 64 heads, Dk and Dv multiples of 64 (Dk <= 576, Dv <= 512).
 //
 // Definitions as in simt_backward.cu ("HySparse MQA sparse attention ...",
 // PaddleFleet pull request 1470, "Core" list: SWA and block-sparse MQA
@@ -47,6 +47,7 @@ struct MmaBwdParams {
   const __nv_bfloat16* dout;
   float* dkey;
   float* dval;
+  float* dq;
 };
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -89,17 +90,47 @@ __device__ __forceinline__ bool selects(const int32_t* row, int topk, int bq, in
   return false;
 }
 
+// Asynchronous 16-byte global -> shared copy (completion: cp_async_wait_all).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
+// q_t and dout_t of one token, all heads, into padded shared-memory tiles
+// (asynchronous copies, all in flight at once; the caller waits and syncs).
+__device__ __forceinline__ void stage_token(__nv_bfloat16* Qs, int KS, __nv_bfloat16* Ds, int VS,
+                                            const __nv_bfloat16* qg, int64_t qrs, int64_t qhs,
+                                            const __nv_bfloat16* dout, int t, int dk, int dv) {
+  const int vq = dk >> 3, vd = dv >> 3;
+  for (int e = threadIdx.x; e < kH * vq; e += kThreads) {
+    const int h = e / vq, c = (e - h * vq) << 3;
+    cp_async16(Qs + h * KS + c, qg + (int64_t)t * qrs + (int64_t)h * qhs + c);
+  }
+  for (int e = threadIdx.x; e < kH * vd; e += kThreads) {
+    const int h = e / vd, c = (e - h * vd) << 3;
+    cp_async16(Ds + h * VS + c, dout + ((int64_t)t * kH + h) * dv + c);
+  }
+}
+
 // 16-byte copy of `rows` rows of `cols` bf16 (cols % 8 == 0) into a padded
 // shared-memory tile; row r of the source starts at src + r * stride.
+// Rows past `rows` (up to zero_rows_to) are zeroed.  Asynchronous for the
+// copied rows: the caller waits (cp_async_wait_all) and syncs.
 __device__ __forceinline__ void copy_rows(__nv_bfloat16* dst, int dst_stride,
                                           const __nv_bfloat16* src, int64_t stride, int rows,
                                           int cols, int zero_rows_to) {
   const int vpr = cols >> 3;  // 16-byte vectors per row
   for (int e = threadIdx.x; e < zero_rows_to * vpr; e += kThreads) {
     const int r = e / vpr, c = (e - r * vpr) << 3;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < rows) v = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)r * stride + c));
-    *reinterpret_cast<uint4*>(dst + r * dst_stride + c) = v;
+    if (r < rows)
+      cp_async16(dst + r * dst_stride + c, src + (int64_t)r * stride + c);
+    else
+      *reinterpret_cast<uint4*>(dst + r * dst_stride + c) = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -145,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_mma_kernel(const MmaBwdP
       const int s1 = min(j1, eos), n = s1 - s0;
       copy_rows(Kt, KS, kg + (int64_t)s0 * P.k_row_stride, P.k_row_stride, n, dk, kKT);
       copy_rows(Vt, VS, vg + (int64_t)s0 * P.v_row_stride, P.v_row_stride, n, dv, kKT);
+      cp_async_wait_all();  // published by the candidate loop's first barrier
       float accK[kMaxNK][4], accV[kMaxNV][4];
 #pragma unroll
       for (int i = 0; i < kMaxNK; ++i) accK[i][0] = accK[i][1] = accK[i][2] = accK[i][3] = 0.f;
@@ -193,23 +225,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_mma_kernel(const MmaBwdP
           const int tt = mem[mi];
           const uint32_t mk = (uint32_t)memmask[mi];
           // q_t and dout_t, all heads, and the token's lse / delta
-          {
-            const int vq = dk >> 3, vd = dv >> 3;
-            for (int e = tid; e < kH * vq; e += kThreads) {
-              const int h = e / vq, c = (e - h * vq) << 3;
-              *reinterpret_cast<uint4*>(Qs + h * KS + c) = __ldg(reinterpret_cast<const uint4*>(
-                  qg + (int64_t)tt * P.q_row_stride + (int64_t)h * P.q_head_stride + c));
-            }
-            for (int e = tid; e < kH * vd; e += kThreads) {
-              const int h = e / vd, c = (e - h * vd) << 3;
-              *reinterpret_cast<uint4*>(Ds + h * VS + c) = __ldg(
-                  reinterpret_cast<const uint4*>(a.dout + ((int64_t)tt * kH + h) * dv + c));
-            }
-            if (tid < kH) {
-              lse_s[tid] = __ldg(a.lse + (int64_t)tt * kH + tid);
-              del_s[tid] = __ldg(a.delta + (int64_t)tt * kH + tid);
-            }
+          stage_token(Qs, KS, Ds, VS, qg, P.q_row_stride, P.q_head_stride, a.dout, tt, dk, dv);
+          if (tid < kH) {
+            lse_s[tid] = __ldg(a.lse + (int64_t)tt * kH + tid);
+            del_s[tid] = __ldg(a.delta + (int64_t)tt * kH + tid);
           }
+          cp_async_wait_all();
           __syncthreads();
           // S^T and dP^T for keys wm*16.. x heads wn*8..
           float sc[4] = {0.f, 0.f, 0.f, 0.f}, dp[4] = {0.f, 0.f, 0.f, 0.f};
@@ -312,6 +333,156 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_mma_kernel(const MmaBwdP
   }
 }
 
+// ---------------------------------------------------------------- dq
+// Query-major: one CTA per token t with q_t and dout_t (all heads) resident;
+// the token's key set in tiles of at most 32 keys that never cross a block
+// (SWA: the window).  Per tile:
+//   S [64 heads x 32 keys] = q_t . K_tile^T,  dP = dout_t . V_tile^T
+//       (16 warps: one 16 x 8 tile each)
+//   dS = P (dP - delta) -> shared memory (bf16, [head][key])
+//   dQ [64 x Dk] += dS . K_tile   (registers: warp w owns heads 16 (w / 4)..
+//       and every fourth 8-column tile from w % 4)
+constexpr int kDS = kKT + kPad;  // row stride of the dS tile
+constexpr int kMaxNQ = 18;       // Dk / 32 n-tiles per warp (Dk <= 576)
+
+inline size_t mma_dq_smem_bytes(int dk, int dv) {
+  const int KS = dk + kPad, VS = dv + kPad;
+  return 2 * ((size_t)kH * KS + (size_t)kH * VS + (size_t)kKT * KS + (size_t)kKT * VS +
+              (size_t)kH * kDS) +
+         4 * 2 * (size_t)kH + 4 * 256;
+}
+
+template <bool kSparse>
+__global__ void __launch_bounds__(kThreads, 1) bwd_dq_mma_kernel(const MmaBwdParams a) {
+  extern __shared__ __align__(16) uint8_t smraw[];
+  __shared__ int nblk;
+  const Problem& P = a.p;
+  const int dk = P.dk, dv = P.dv, KS = dk + kPad, VS = dv + kPad;
+  __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(smraw);  // [kH][KS]
+  __nv_bfloat16* Ds = Qs + kH * KS;                              // [kH][VS]
+  __nv_bfloat16* Kt = Ds + kH * VS;                              // [kKT][KS]
+  __nv_bfloat16* Vt = Kt + kKT * KS;                             // [kKT][VS]
+  __nv_bfloat16* Sd = Vt + kKT * VS;                             // [kH][kDS] dS
+  float* lse_s = reinterpret_cast<float*>(Sd + kH * kDS);
+  float* del_s = lse_s + kH;
+  int* blist = reinterpret_cast<int*>(del_s + kH);               // [256]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tig = lane & 3;
+  const int wm = warp >> 2;  // 16-head tile
+  const int wn = warp & 3;   // 8-key tile (scores) / n-tile phase (dq)
+  const int nQ = dk >> 5;
+  const float scale = P.scale;
+  const uint32_t kt_base = (uint32_t)__cvta_generic_to_shared(Kt);
+  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(P.q);
+  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(P.k);
+  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(P.v);
+  for (int t = blockIdx.x; t < P.total_tokens; t += gridDim.x) {
+    int bos, eos;
+    if (!find_doc(P.cu_seqlens, P.num_docs, P.total_tokens, P.max_seqlen, t, bos, eos, P.status))
+      continue;
+    if (kSparse && tid == 0) {
+      const int bq = (t - bos) / a.B;
+      const int32_t* row = a.idx + (int64_t)t * a.topk;
+      int nb = 0;
+      bool bad = false;
+      for (int sl = 0; sl < a.topk; ++sl) {
+        int b;
+        if (entry_used(row, sl, bq, b)) blist[nb++] = b;
+        else if (b >= 0) bad = true;
+      }
+      if (bad) record_status(P.status, HS_ERR_INVALID_INDEX);
+      nblk = nb;
+    }
+    stage_token(Qs, KS, Ds, VS, qg, P.q_row_stride, P.q_head_stride, a.dout, t, dk, dv);
+    if (tid < kH) {
+      lse_s[tid] = __ldg(a.lse + (int64_t)t * kH + tid);
+      del_s[tid] = __ldg(a.delta + (int64_t)t * kH + tid);
+    }
+    cp_async_wait_all();
+    float acc[kMaxNQ][4];
+#pragma unroll
+    for (int i = 0; i < kMaxNQ; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    __syncthreads();
+    const int nseg = kSparse ? nblk : 1;
+    for (int sg = 0; sg < nseg; ++sg) {
+      int lo, hi;
+      if (kSparse) {
+        lo = bos + blist[sg] * a.B;
+        hi = min(min(lo + a.B, eos), t + 1);
+      } else {
+        lo = max(bos, t - a.window + 1);
+        hi = t + 1;
+      }
+      for (int j0 = lo; j0 < hi; j0 += kKT) {
+        const int n = min(kKT, hi - j0);
+        copy_rows(Kt, KS, kg + (int64_t)j0 * P.k_row_stride, P.k_row_stride, n, dk, kKT);
+        copy_rows(Vt, VS, vg + (int64_t)j0 * P.v_row_stride, P.v_row_stride, n, dv, kKT);
+        cp_async_wait_all();
+        __syncthreads();
+        float sc[4] = {0.f, 0.f, 0.f, 0.f}, dp[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+          const __nv_bfloat16* qa = Qs + (wm * 16 + g) * KS + 2 * tig;
+          const __nv_bfloat16* kb = Kt + (wn * 8 + g) * KS + 2 * tig;
+          for (int k0 = 0; k0 < dk; k0 += 16) {
+            const uint32_t af[4] = {lds32(qa + k0), lds32(qa + 8 * KS + k0), lds32(qa + k0 + 8),
+                                    lds32(qa + 8 * KS + k0 + 8)};
+            mma16816(sc, af, lds32(kb + k0), lds32(kb + k0 + 8));
+          }
+          const __nv_bfloat16* da = Ds + (wm * 16 + g) * VS + 2 * tig;
+          const __nv_bfloat16* vb = Vt + (wn * 8 + g) * VS + 2 * tig;
+          for (int k0 = 0; k0 < dv; k0 += 16) {
+            const uint32_t af[4] = {lds32(da + k0), lds32(da + 8 * VS + k0), lds32(da + k0 + 8),
+                                    lds32(da + 8 * VS + k0 + 8)};
+            mma16816(dp, af, lds32(vb + k0), lds32(vb + k0 + 8));
+          }
+        }
+        {
+          const int h0 = wm * 16 + g, c0 = wn * 8 + 2 * tig;
+          float dsv[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int head = h0 + ((q & 2) ? 8 : 0), key = c0 + (q & 1);
+            const float pr = key < n ? expf(sc[q] * scale - lse_s[head]) : 0.f;
+            dsv[q] = pr * (dp[q] - del_s[head]);
+          }
+          *reinterpret_cast<uint32_t*>(Sd + h0 * kDS + c0) = pack_bf16(dsv[0], dsv[1]);
+          *reinterpret_cast<uint32_t*>(Sd + (h0 + 8) * kDS + c0) = pack_bf16(dsv[2], dsv[3]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int ks = 0; ks < kKT / 16; ++ks) {
+          const __nv_bfloat16* sa = Sd + (wm * 16 + g) * kDS + ks * 16 + 2 * tig;
+          const uint32_t af[4] = {lds32(sa), lds32(sa + 8 * kDS), lds32(sa + 8),
+                                  lds32(sa + 8 * kDS + 8)};
+          const uint32_t krow = kt_base + (uint32_t)((ks * 16 + (lane & 15)) * KS) * 2u;
+#pragma unroll
+          for (int i = 0; i < kMaxNQ; ++i) {
+            if (i < nQ) {
+              uint32_t b0, b1;
+              ldsm_x2_trans(b0, b1, krow + (uint32_t)((wn + 4 * i) * 16));
+              mma16816(acc[i], af, b0, b1);
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    {
+      const int h0 = wm * 16 + g;
+      float* dq0 = a.dq + ((int64_t)t * kH + h0) * dk;
+#pragma unroll
+      for (int i = 0; i < kMaxNQ; ++i) {
+        if (i < nQ) {
+          const int col = (wn + 4 * i) * 8 + 2 * tig;
+          *reinterpret_cast<float2*>(dq0 + col) = make_float2(scale * acc[i][0], scale * acc[i][1]);
+          *reinterpret_cast<float2*>(dq0 + 8 * dk + col) =
+              make_float2(scale * acc[i][2], scale * acc[i][3]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace
 
 bool mma_backward_supported(const Problem& p) {
@@ -320,7 +491,28 @@ bool mma_backward_supported(const Problem& p) {
          p.dk <= 64 * kMaxNK && p.dv % 64 == 0 && p.dv >= 64 && p.dv <= 64 * kMaxNV &&
          al16(p.q) && al16(p.k) && al16(p.v) && p.q_row_stride % 8 == 0 &&
          p.q_head_stride % 8 == 0 && p.k_row_stride % 8 == 0 && p.v_row_stride % 8 == 0 &&
-         mma_dkdv_smem_bytes(p.dk, p.dv) <= 227 * 1024;
+         mma_dkdv_smem_bytes(p.dk, p.dv) <= 227 * 1024 && mma_dq_smem_bytes(p.dk, p.dv) <= 227 * 1024;
+}
+
+cudaError_t launch_mma_dq(const BwdArgs& b, bool sparse, const float* delta, cudaStream_t s) {
+  MmaBwdParams a;
+  a.p = b.p;
+  a.idx = b.idx;
+  a.topk = b.topk;
+  a.B = b.block_size;
+  a.window = b.window;
+  a.lse = b.lse;
+  a.delta = delta;
+  a.dout = static_cast<const __nv_bfloat16*>(b.dout);
+  a.dkey = nullptr;
+  a.dval = nullptr;
+  a.dq = b.dq;
+  const size_t bytes = mma_dq_smem_bytes(b.p.dk, b.p.dv);
+  auto kern = sparse ? bwd_dq_mma_kernel<true> : bwd_dq_mma_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  kern<<<b.p.total_tokens, kThreads, bytes, s>>>(a);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_mma_dkdv(const BwdArgs& b, bool sparse, const float* delta, cudaStream_t s) {
@@ -335,6 +527,7 @@ cudaError_t launch_mma_dkdv(const BwdArgs& b, bool sparse, const float* delta, c
   a.dout = static_cast<const __nv_bfloat16*>(b.dout);
   a.dkey = b.dkey;
   a.dval = b.dval;
+  a.dq = nullptr;
   const size_t bytes = mma_dkdv_smem_bytes(b.p.dk, b.p.dv);
   auto kern = sparse ? bwd_dkdv_mma_kernel<true> : bwd_dkdv_mma_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);

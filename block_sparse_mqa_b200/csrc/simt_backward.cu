@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(const BwdParams a, i
 constexpr size_t kMaxSmem = 227 * 1024;
 
 template <typename T, bool kSparse>
-cudaError_t launch_typed(BwdParams a, bool dkdv, cudaStream_t s) {
+cudaError_t launch_typed(BwdParams a, bool cuda_core_passes, cudaStream_t s) {
   const Problem& P = a.p;
   const int NT = P.total_tokens, H = P.num_heads;
   const int pairs = NT * H;
@@ -406,8 +406,9 @@ cudaError_t launch_typed(BwdParams a, bool dkdv, cudaStream_t s) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  // dq: the largest head group (and key tile) whose staging fits
-  {
+  // dq: the largest head group (and key tile) whose staging fits (unless the
+  // caller runs the tensor-core passes instead)
+  if (cuda_core_passes) {
     int G = 16, KT = 16;
     const size_t ints = 256 * sizeof(int);
     while (G > 1 && dq_smem_floats(G, KT, P.dk, P.dv) * 4 + ints > kMaxSmem) G >>= 1;
@@ -425,7 +426,7 @@ cudaError_t launch_typed(BwdParams a, bool dkdv, cudaStream_t s) {
   }
   // dk, dv: key tiles of at most kKeyTile keys (unless the caller runs the
   // tensor-core key-major pass instead)
-  if (dkdv) {
+  if (cuda_core_passes) {
     int G = 16, KT = kKeyTile;
     const size_t ints = 2 * kThreads * sizeof(int);
     while (KT > 4 && dkdv_smem_floats(G, KT, P.dk, P.dv) * 4 + ints > kMaxSmem) KT >>= 1;
@@ -470,6 +471,8 @@ cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, cudaStream_t s) 
     cudaError_t e = sparse ? launch_typed<__nv_bfloat16, true>(a, !mma, s)
                            : launch_typed<__nv_bfloat16, false>(a, !mma, s);
     if (e != cudaSuccess || !mma) return e;
+    e = launch_mma_dq(b, sparse, a.delta, s);
+    if (e != cudaSuccess) return e;
     return launch_mma_dkdv(b, sparse, a.delta, s);
   }
   return sparse ? launch_typed<float, true>(a, true, s) : launch_typed<float, false>(a, true, s);
