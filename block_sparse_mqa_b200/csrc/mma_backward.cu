@@ -11,16 +11,20 @@
 // Why warp-level MMAs here: a key tile's dk and dv accumulators (keys x
 // (Dk + Dv) fp32) do not fit the 512 TMEM columns beside the score tiles at
 // Dk 576 / Dv 512, while registers spread over 16 warps hold them for a tile
-// of 32 keys.  One CTA per 32-key tile (split at document boundaries); the
-// tile's K and V rows stay in shared memory; the queries whose key set meets
-// the tile are found by scanning candidate idx rows (or the window) and are
-// visited in ascending order.  Per member token t (all 64 heads):
+// of 32 keys.  A cluster of four CTAs per 32-key tile (split at document
+// boundaries); each keeps the tile's K and V rows in shared memory, finds the
+// queries whose key set meets the tile by scanning candidate idx rows (or the
+// window), takes every fourth of them in ascending order, and the four
+// partial sums are added in rank order through distributed shared memory
+// (a tile every query selects, such as a document's first block, is then
+// spread over four SMs).  Per member token t (all 64 heads):
 //   S^T [32 keys x 64 heads]  = K_tile . q_t^T      (each warp one 16x8 tile)
 //   dP^T[32 x 64]             = V_tile . dout_t^T
 //   P^T, dS^T (bf16)          -> shared memory
 //   dK[32 x Dk] += dS^T . q_t,  dV[32 x Dv] += P^T . dout_t   (registers)
 // Sums run in a fixed order: results are deterministic.
 
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -30,7 +34,10 @@
 namespace hs {
 namespace {
 
+namespace cg = cooperative_groups;
+
 constexpr int kThreads = 512;   // 16 warps
+constexpr int kCluster = 4;     // CTAs sharing one key tile (dk / dv pass)
 constexpr int kKT = 32;         // keys per tile (two m16 tiles)
 constexpr int kH = 64;          // heads
 constexpr int kPad = 8;         // bf16 elements of row padding (16 bytes)
@@ -168,7 +175,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_mma_kernel(const MmaBwdP
   const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(P.q);
   const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(P.k);
   const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(P.v);
-  for (int tile = blockIdx.x; tile * kKT < NT; tile += gridDim.x) {
+  // The CTAs of a cluster share one key tile: each scans every candidate
+  // (so all see the same member list) and takes every csize-th member; their
+  // partial sums are added in rank order through distributed shared memory.
+  cg::cluster_group cl = cg::this_cluster();
+  const int crank = (int)cl.block_rank(), csize = (int)cl.num_blocks();
+  const int ncl = gridDim.x / csize;
+  for (int tile = blockIdx.x / csize; tile * kKT < NT; tile += ncl) {
     const int j1 = min(NT, tile * kKT + kKT);
     for (int s0 = tile * kKT; s0 < j1;) {  // one document segment at a time
       int bos, eos;
@@ -221,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_mma_kernel(const MmaBwdP
           memmask[pos] = (int)mask;
         }
         __syncthreads();
-        for (int mi = 0; mi < nm; ++mi) {
+        for (int mi = crank; mi < nm; mi += csize) {
           const int tt = mem[mi];
           const uint32_t mk = (uint32_t)memmask[mi];
           // q_t and dout_t, all heads, and the token's lse / delta
@@ -299,35 +312,43 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_mma_kernel(const MmaBwdP
           __syncthreads();
         }
       }
-      // this segment's rows of dk (scaled) and dv
+      // this CTA's partial sums -> its shared memory (the q / dout staging
+      // area is free: [kKT][Dk + Dv] fp32); the cluster adds them in rank
+      // order, rank r writing keys r, r + csize, ... of the segment
       {
-        const int r0 = wm * 16 + g;
+        const int W = dk + dv, r0 = wm * 16 + g;
+        float* part = reinterpret_cast<float*>(Qs);
 #pragma unroll
         for (int i = 0; i < kMaxNK; ++i) {
           if (i < nK) {
             const int col = (wn + 8 * i) * 8 + 2 * tig;
-            if (r0 < n)
-              *reinterpret_cast<float2*>(a.dkey + (int64_t)(s0 + r0) * dk + col) =
-                  make_float2(scale * accK[i][0], scale * accK[i][1]);
-            if (r0 + 8 < n)
-              *reinterpret_cast<float2*>(a.dkey + (int64_t)(s0 + r0 + 8) * dk + col) =
-                  make_float2(scale * accK[i][2], scale * accK[i][3]);
+            *reinterpret_cast<float2*>(part + r0 * W + col) = make_float2(accK[i][0], accK[i][1]);
+            *reinterpret_cast<float2*>(part + (r0 + 8) * W + col) =
+                make_float2(accK[i][2], accK[i][3]);
           }
         }
 #pragma unroll
         for (int i = 0; i < kMaxNV; ++i) {
           if (i < nV) {
-            const int col = (wn + 8 * i) * 8 + 2 * tig;
-            if (r0 < n)
-              *reinterpret_cast<float2*>(a.dval + (int64_t)(s0 + r0) * dv + col) =
-                  make_float2(accV[i][0], accV[i][1]);
-            if (r0 + 8 < n)
-              *reinterpret_cast<float2*>(a.dval + (int64_t)(s0 + r0 + 8) * dv + col) =
-                  make_float2(accV[i][2], accV[i][3]);
+            const int col = dk + (wn + 8 * i) * 8 + 2 * tig;
+            *reinterpret_cast<float2*>(part + r0 * W + col) = make_float2(accV[i][0], accV[i][1]);
+            *reinterpret_cast<float2*>(part + (r0 + 8) * W + col) =
+                make_float2(accV[i][2], accV[i][3]);
           }
         }
+        cl.sync();
+        const int mine = n > crank ? (n - crank + csize - 1) / csize : 0;
+        for (int e = tid; e < mine * W; e += kThreads) {
+          const int kk = crank + (e / W) * csize, col = e - (e / W) * W;
+          float sum = 0.f;
+          for (int rr = 0; rr < csize; ++rr) sum += cl.map_shared_rank(part, rr)[kk * W + col];
+          if (col < dk)
+            a.dkey[(int64_t)(s0 + kk) * dk + col] = scale * sum;
+          else
+            a.dval[(int64_t)(s0 + kk) * dv + (col - dk)] = sum;
+        }
+        cl.sync();  // no CTA reuses its shared memory while another still reads it
       }
-      __syncthreads();
       s0 = s1;
     }
   }
@@ -532,9 +553,29 @@ cudaError_t launch_mma_dkdv(const BwdArgs& b, bool sparse, const float* delta, c
   auto kern = sparse ? bwd_dkdv_mma_kernel<true> : bwd_dkdv_mma_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
-  const int grid = (b.p.total_tokens + kKT - 1) / kKT;
-  kern<<<grid, kThreads, bytes, s>>>(a);
-  return cudaGetLastError();
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+  if (e != cudaSuccess) return e;
+  const int tiles = (b.p.total_tokens + kKT - 1) / kKT;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // clusters of kCluster CTAs when the device can place them, else single CTAs
+  int nclusters = 0;
+  cfg.gridDim = dim3(tiles * kCluster);
+  if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters < 1) {
+    (void)cudaGetLastError();
+    attr[0].val.clusterDim.x = 1;
+    cfg.gridDim = dim3(tiles);
+  }
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 }  // namespace hs
