@@ -453,7 +453,10 @@ def run_backward(inp, wl, step, cu, pk, reps=2):
         fl = 2.0 * H * (3 * wl.dk + 2 * wl.dv) * pairs[name]
         tf = fl / (ms / 1e3) / 1e12
         res[name] = {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / pk["bf16_tflops"],
-                     "algorithmic_flops": fl, "path": "simt", "calls_timed": reps}
+                     "algorithmic_flops": fl, "calls_timed": reps,
+                     "path": {hs.HS_PATH_MMA: "mma.sync", hs.HS_PATH_SIMT: "simt"}.get(
+                         hs.path(hs.HS_OP_SPARSE_MQA_BWD if name == "sparse" else hs.HS_OP_SWA_MQA_BWD,
+                                 wl.dtype, H, wl.dk, wl.dv, wl.block_size), "other")}
     hs.poll_status(inp.q.device)
     return res
 

@@ -165,6 +165,8 @@ int hs_path(int op, hs_dtype dtype, int num_heads, int dk, int dv, int block_siz
       return HS_PATH_SIMT;
     case HS_OP_SPARSE_MQA_BWD:
     case HS_OP_SWA_MQA_BWD:
+      if (!g_force_simt.load() && hs::mma_backward_shape_ok(dtype, num_heads, dk, dv))
+        return HS_PATH_MMA;
       return HS_PATH_SIMT;
     case HS_OP_SPARSE_MQA:
     case HS_OP_SWA_MQA:
@@ -382,7 +384,7 @@ static hs_status backward_common(hs::BwdArgs& a, bool sparse, const void* q, int
   a.workspace = workspace;
   r = status_ptr(&a.p.status);
   if (r != HS_OK) return r;
-  return launched(hs::launch_simt_backward(a, sparse, stream),
+  return launched(hs::launch_simt_backward(a, sparse, !g_force_simt.load(), stream),
                   sparse ? "simt sparse attention backward" : "simt swa attention backward");
 }
 

@@ -506,10 +506,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_mma_kernel(const MmaBwdPar
 
 }  // namespace
 
+bool mma_backward_shape_ok(hs_dtype dtype, int num_heads, int dk, int dv) {
+  return dtype == HS_BF16 && num_heads == kH && dk % 64 == 0 && dk >= 64 && dk <= 64 * kMaxNK &&
+         dv % 64 == 0 && dv >= 64 && dv <= 64 * kMaxNV;
+}
+
 bool mma_backward_supported(const Problem& p) {
   auto al16 = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; };
-  return p.dtype == HS_BF16 && p.num_heads == kH && p.dk % 64 == 0 && p.dk >= 64 &&
-         p.dk <= 64 * kMaxNK && p.dv % 64 == 0 && p.dv >= 64 && p.dv <= 64 * kMaxNV &&
+  return mma_backward_shape_ok(p.dtype, p.num_heads, p.dk, p.dv) &&
          al16(p.q) && al16(p.k) && al16(p.v) && p.q_row_stride % 8 == 0 &&
          p.q_head_stride % 8 == 0 && p.k_row_stride % 8 == 0 && p.v_row_stride % 8 == 0 &&
          mma_dkdv_smem_bytes(p.dk, p.dv) <= 227 * 1024 && mma_dq_smem_bytes(p.dk, p.dv) <= 227 * 1024;

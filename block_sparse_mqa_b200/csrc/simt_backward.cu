@@ -449,7 +449,7 @@ size_t simt_backward_workspace(int total_tokens, int num_heads) {
   return (size_t)2 * total_tokens * num_heads * sizeof(float);
 }
 
-cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, cudaStream_t s) {
+cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, bool allow_mma, cudaStream_t s) {
   BwdParams a{};
   a.p = b.p;
   a.idx = b.idx;
@@ -467,7 +467,7 @@ cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, cudaStream_t s) 
   a.delta = static_cast<float*>(b.workspace);
   a.dsink_part = a.delta + (size_t)b.p.total_tokens * b.p.num_heads;
   if (b.p.dtype == HS_BF16) {
-    const bool mma = mma_backward_supported(b.p);
+    const bool mma = allow_mma && mma_backward_supported(b.p);
     cudaError_t e = sparse ? launch_typed<__nv_bfloat16, true>(a, !mma, s)
                            : launch_typed<__nv_bfloat16, false>(a, !mma, s);
     if (e != cudaSuccess || !mma) return e;

@@ -40,6 +40,7 @@ HS_OP_SWA_MQA_BWD = 5
 
 HS_PATH_SIMT = 0
 HS_PATH_TCGEN05 = 1
+HS_PATH_MMA = 2
 
 # every symbol include/hs.h declares
 EXPORTS = (

@@ -99,8 +99,10 @@ typedef enum hs_op {
 
 /* Kernel family a call will use, as returned by hs_path(). */
 typedef enum hs_kernel_path {
-  HS_PATH_SIMT = 0,   /* CUDA-core kernel: fp32 inputs, unusual shapes    */
-  HS_PATH_TCGEN05 = 1 /* tcgen05 tensor-core kernel (TMEM accumulators)   */
+  HS_PATH_SIMT = 0,    /* CUDA-core kernel: fp32 inputs, unusual shapes    */
+  HS_PATH_TCGEN05 = 1, /* tcgen05 tensor-core kernel (TMEM accumulators)   */
+  HS_PATH_MMA = 2      /* warp-level tensor-core MMAs (register accumulators;
+                          the backward, whose accumulators exceed TMEM)    */
 } hs_kernel_path;
 
 /*
@@ -240,7 +242,10 @@ hs_status hs_swa_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_str
  *              HS_ERR_WORKSPACE before any device work.
  * idx entries follow the forward's rule; offending entries are skipped and
  * reported as HS_ERR_INVALID_INDEX.  Results are deterministic (every sum
- * runs in a fixed order).
+ * runs in a fixed order).  bf16 inputs with 64 heads and Dk, Dv multiples of
+ * 64 run on warp-level tensor-core MMAs (hs_path: HS_PATH_MMA); other inputs
+ * on CUDA cores.  The call launches a four-CTA cluster kernel and falls back
+ * to single CTAs where the device cannot place the cluster.
  */
 hs_status hs_sparse_mqa_bwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
                             const void* k, int64_t k_row_stride,

@@ -118,7 +118,9 @@ def test_backward_rejects_bad_arguments():
     need = L.hs_workspace_size(hs.HS_OP_SPARSE_MQA_BWD, T, 1, 100, H, 576, 512, hs.HS_BF16, 64)
     assert need == 8 * T * H
     assert L.hs_workspace_size(hs.HS_OP_SWA_MQA_BWD, T, 1, 100, H, 576, 512, hs.HS_BF16, 64) == need
-    assert L.hs_path(hs.HS_OP_SPARSE_MQA_BWD, hs.HS_BF16, H, 576, 512, 64) == hs.HS_PATH_SIMT
+    assert L.hs_path(hs.HS_OP_SPARSE_MQA_BWD, hs.HS_BF16, H, 576, 512, 64) == hs.HS_PATH_MMA
+    assert L.hs_path(hs.HS_OP_SWA_MQA_BWD, hs.HS_F32, H, 576, 512, 64) == hs.HS_PATH_SIMT
+    assert L.hs_path(hs.HS_OP_SWA_MQA_BWD, hs.HS_BF16, 20, 80, 48, 64) == hs.HS_PATH_SIMT
     args = [p, 64 * 576, 576, p, 576, p, 512, p, 1, T, 100, H, 576, 512, hs.HS_BF16, 0.0]
     tail = [p, p, p, p, p, p, None]  # out, lse, dout, dq, dk, dv, dsink
     # sparse: bad topk / idx / block, missing gradient outputs, workspace

@@ -118,6 +118,18 @@ def test_backward_tensor_core_variants(B, K, W, dk, dv):
         run_backward(docs, 64, dk, dv, torch.bfloat16, kind, B=B, K=K, W=W, seed=3)
 
 
+
+def test_backward_paths_and_forced_cuda_cores():
+    assert hs.path(hs.HS_OP_SPARSE_MQA_BWD, torch.bfloat16, 64, 576, 512, 64) == hs.HS_PATH_MMA
+    assert hs.path(hs.HS_OP_SWA_MQA_BWD, torch.float32, 64, 576, 512, 64) == hs.HS_PATH_SIMT
+    hs.set_force_simt(True)
+    try:
+        assert hs.path(hs.HS_OP_SPARSE_MQA_BWD, torch.bfloat16, 64, 576, 512, 64) == hs.HS_PATH_SIMT
+        for kind in ("sparse", "swa"):
+            run_backward([130, 64, 1, 257], 64, 576, 512, torch.bfloat16, kind, seed=1)
+    finally:
+        hs.set_force_simt(False)
+
 def test_backward_other_dims():
     # Dk != Dv, not multiples of 64; several head groups with a partial last one
     run_backward([120, 88], 20, 80, 48, torch.float32, "sparse", B=16, K=3, seed=4)
