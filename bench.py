@@ -54,7 +54,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the (separately timed) backward of the two attention steps")
-    ap.add_argument("--cpu-rows", type=int, default=1536,
+    ap.add_argument("--cpu-rows", type=int, default=3072,
                     help="query rows of the oracle sample (cpu_baseline / reference arm)")
     return ap.parse_args()
 
@@ -72,6 +72,10 @@ def ncu_traffic(kernel):
     if hashlib.sha256(src).hexdigest() != rec["sha256"]:
         return None
     return rec["bytes"]
+
+
+NOMINAL_BF16_TFLOPS = 2250.0   # dense bf16, per GPU (context only)
+NOMINAL_HBM_GBS = 8000.0
 
 
 def peaks():
@@ -218,8 +222,8 @@ def run_cpu_baseline(wl, rows_n, steps=1):
     used, aff, blas = cpu_cores()
     return {"value": len(rows) * steps / dt, "unit": UNIT, "cores": used, "kind": "oracle",
             "sample": "%d query rows of %s (all four steps, float64 NumPy), %d step(s), %.1f s; "
-                      "affinity %d cores, BLAS threads %d" % (len(rows), wl.name, steps, dt, aff,
-                                                              blas)}
+                      "os.cpu_count() %d, affinity %d cores, BLAS threads %d" % (
+                          len(rows), wl.name, steps, dt, os.cpu_count() or 0, aff, blas)}
 
 
 # ---------------------------------------------------------------------------
@@ -369,12 +373,19 @@ def run_ours(args, wl, world, rank):
     for ph in ("score", "sparse", "swa"):
         tf = flops[ph] / (avg[ph] / 1e3) / 1e12
         kernels[ph] = {"ms": avg[ph], "tflops": tf, "frac_of_bf16_peak": tf / pk["bf16_tflops"],
+                       "frac_of_nominal_bf16": tf / NOMINAL_BF16_TFLOPS,
                        "algorithmic_flops": flops[ph],
                        "path": "tcgen05" if hs.path(
                            {"score": 0, "sparse": 2, "swa": 3}[ph], wl.dtype, H, wl.dk, wl.dv,
                            wl.block_size) == hs.HS_PATH_TCGEN05 else "simt"}
     sel_gbs = sel_bytes / (avg["select"] / 1e3) / 1e9
+    # gather traffic of the sparse step: every valid (query, key) pair moves one
+    # K row and one V row from L2 to an SM (the unique KV is only T rows)
+    kernels["sparse"]["gather_bytes_l2_to_sm"] = 2.0 * (wl.dk + wl.dv) * flops["sparse"] / (
+        2.0 * H * (wl.dk + wl.dv))
+    kernels["sparse"]["unique_kv_bytes"] = 2.0 * (wl.dk + wl.dv) * wl.total_tokens
     kernels["select"] = {"ms": avg["select"], "gbs": sel_gbs, "frac_of_hbm": sel_gbs / pk["hbm_gbs"],
+                         "frac_of_nominal_hbm": sel_gbs / NOMINAL_HBM_GBS,
                          "algorithmic_bytes": sel_bytes, "path": "simt"}
     dom = max(("score", "sparse", "swa"), key=lambda ph: avg[ph])
     roof = {"bound": "tensor", "achieved": kernels[dom]["tflops"], "peak": pk["bf16_tflops"],
