@@ -474,42 +474,76 @@ def run_backward(inp, wl, step, cu, pk, reps=2):
 
 def run_e2e(inp, wl, step, steps, world):
     """Same metric through the public API with host buffers: every step copies
-    the inputs from pinned host memory, runs the four calls and copies the
-    outputs back; all inside the timed region."""
+    its inputs from pinned host memory, runs the four calls and copies its
+    outputs back, all inside the timed region.  Consecutive steps overlap as
+    in a serving loop: two device buffer sets, and the input copies, the
+    kernels and the output copies on three streams ordered by events (step
+    s + 1's inputs and step s - 1's outputs cross PCIe while step s runs)."""
+    import dataclasses
     dev = inp.q.device
     hq = inp.q.cpu().pin_memory()
     hk = inp.k.cpu().pin_memory()
     hv = inp.v.cpu().pin_memory()
     hsink = inp.sink.cpu().pin_memory()
     hcu = inp.cu_seqlens.cpu().pin_memory()
-    outs = [step.out, step.lse, step.wout, step.wlse, step.idx]
-    houts = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    inp2 = dataclasses.replace(inp, q=torch.empty_like(inp.q), k=torch.empty_like(inp.k),
+                               v=torch.empty_like(inp.v), sink=torch.empty_like(inp.sink),
+                               cu_seqlens=torch.empty_like(inp.cu_seqlens))
+    sets = [(inp, step), (inp2, Step(inp2, wl))]
+    outs = [[st.out, st.lse, st.wout, st.wlse, st.idx] for _, st in sets]
+    houts = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in oo] for oo in outs]
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsink, hcu))
-    d2h = sum(t.numel() * t.element_size() for t in houts)
+    d2h = sum(t.numel() * t.element_size() for t in houts[0])
+    s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_run = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        inp.q.copy_(hq, non_blocking=True)
-        inp.k.copy_(hk, non_blocking=True)
-        inp.v.copy_(hv, non_blocking=True)
-        inp.sink.copy_(hsink, non_blocking=True)
-        inp.cu_seqlens.copy_(hcu, non_blocking=True)
-        step.run()
-        for o, h in zip(outs, houts):
-            h.copy_(o, non_blocking=True)
+    def issue(n):
+        k = n % 2
+        ip, st = sets[k]
+        with torch.cuda.stream(s_in):
+            if n >= 2:
+                s_in.wait_event(ev_run[k])  # step n - 2 has read this set's inputs
+            ip.q.copy_(hq, non_blocking=True)
+            ip.k.copy_(hk, non_blocking=True)
+            ip.v.copy_(hv, non_blocking=True)
+            ip.sink.copy_(hsink, non_blocking=True)
+            ip.cu_seqlens.copy_(hcu, non_blocking=True)
+            ev_in[k].record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(ev_in[k])
+            if n >= 2:
+                s_run.wait_event(ev_out[k])  # step n - 2's outputs have left this set
+            st.run()
+            ev_run[k].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_run[k])
+            for o, h in zip(outs[k], houts[k]):
+                h.copy_(o, non_blocking=True)
+            ev_out[k].record(s_out)
 
-    one()
+    for n in range(2):
+        issue(n)
     torch.cuda.synchronize()
     barrier(world)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        one()
-    b.record()
+    cur = torch.cuda.current_stream(dev)
+    a.record(cur)
+    for st_ in (s_in, s_run, s_out):
+        st_.wait_event(a)
+    for n in range(steps):
+        issue(n + 2)
+    for k in range(2):
+        cur.wait_event(ev_out[k])
+    b.record(cur)
     torch.cuda.synchronize()
+    hs.poll_status(dev)
     ms = max_over_ranks(a.elapsed_time(b), world) / steps
     return {"value": wl.total_tokens * world / (ms / 1e3), "unit": UNIT,
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms,
+            "overlap": "steps pipelined: H2D, kernels and D2H on three streams, two buffer sets"}
 
 
 # ---------------------------------------------------------------------------
