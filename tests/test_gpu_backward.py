@@ -130,6 +130,32 @@ def test_backward_paths_and_forced_cuda_cores():
     finally:
         hs.set_force_simt(False)
 
+
+def test_backward_with_v_aliasing_k():
+    """v = k[:, :Dv] (the absorbed-MLA latent slice, a strided view of k): the
+    call returns the gradients of its k and v arguments separately; the
+    caller adds dv into the first Dv columns of dk."""
+    docs = [200, 133]
+    T, H, dk, dv = sum(docs), 64, 576, 512
+    inp = synth.make_inputs(T, H, dk, dv, dtype=torch.bfloat16, seed=21, device=DEV,
+                            doc_lengths=docs)
+    v = inp.k[:, :dv]
+    assert v.stride(0) == dk
+    q, k, s = _np(inp.q), _np(inp.k), _np(inp.sink)
+    cu = inp.cu_seqlens.cpu().tolist()
+    dout = _dout(T, H, dv, torch.bfloat16, 21)
+    ref_idx = O.select_topk(O.block_score(q, k, cu, 64)["block_score"], cu, 64, 4)
+    idx = torch.as_tensor(np.ascontiguousarray(ref_idx, dtype=np.int32), device=DEV)
+    out, lse = hs.hs_sparse_mqa_fwd(inp.q, inp.k, v, idx, inp.cu_seqlens, inp.max_seqlen, 64,
+                                    inp.sink)
+    g = hs.hs_sparse_mqa_bwd(inp.q, inp.k, v, idx, inp.cu_seqlens, inp.max_seqlen, 64, out, lse,
+                             dout, inp.sink)
+    torch.cuda.synchronize()
+    hs.poll_status()
+    ref = OB.sparse_mqa_bwd(q, k, k[:, :dv], _np(dout), ref_idx, cu, 64, sink=s)
+    for gpu, name in zip(g, ("dq", "dk", "dv", "dsink")):
+        check_grad(gpu, ref[name], torch.bfloat16, "aliased " + name)
+
 def test_backward_other_dims():
     # Dk != Dv, not multiples of 64; several head groups with a partial last one
     run_backward([120, 88], 20, 80, 48, torch.float32, "sparse", B=16, K=3, seed=4)
