@@ -2,7 +2,9 @@
 
 This package is the plain, slow, float64 definition of the four forward steps
 (block scoring, top-k block selection, block-sparse MQA attention and
-sliding-window MQA attention) that the CUDA library is checked against.
+sliding-window MQA attention), of the full layer's forward that emits the
+block scores with its attention output, and of the backward of the two
+attention steps, which the CUDA library is checked against.
 
 It is test infrastructure: only the test-suite, the smoke check in
 ``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import it.
@@ -11,7 +13,8 @@ The CUDA product path never imports it and shares no code with it.
 Modules
 -------
 hysparse
-    Vectorised NumPy float64 implementation of the four steps.
+    Vectorised NumPy float64 implementation of the four steps and of the
+    full layer's fused forward (``full_layer_fwd``).
 backward
     The gradient of the two attention steps (dq, dk, dv, sink gradient).
 loops
@@ -32,4 +35,5 @@ from .hysparse import (  # noqa: F401
     sparse_mqa_fwd,
     swa_mqa_fwd,
     dense_causal_fwd,
+    full_layer_fwd,
 )

@@ -66,6 +66,7 @@ __all__ = [
     "sparse_mqa_fwd",
     "swa_mqa_fwd",
     "dense_causal_fwd",
+    "full_layer_fwd",
 ]
 
 
@@ -349,3 +350,63 @@ def dense_causal_fwd(q, k, v, cu_seqlens, sink=None, scale=None, rows=None):
         return np.arange(bos, t + 1, dtype=np.int64)
 
     return _attend_rows(q, k, v, cu_seqlens, sink, scale, rows, keys)
+
+
+# ---------------------------------------------------------------------------
+# the full layer's forward with its block scores (one pass over the logits)
+# ---------------------------------------------------------------------------
+
+def full_layer_fwd(q, k, v, cu_seqlens, block_size: int, scale=None, rows=None):
+    """Forward of the full-attention layer that also scores the key blocks
+    ([HS] "Core": FA4-fused block scoring, "HySparse full layer" bullet of
+    the Copilot overview: the full layer produces the shared KV and the
+    block indices; per-file table, ``block_score_fa4.py``: the block scorer
+    is that layer's flash-attention forward emitting a scaled block_logit;
+    [REV]: its PyLayer saves ``out`` and ``lse``).
+
+    Per query t of document [bos, eos) and head h, over the causal keys
+    j in [bos, t] with s_j = scale * <q[t,h], k[j]> and no sink::
+
+        lse[t,h]          = log sum_j exp(s_j)
+        out[t,h]          = sum_j exp(s_j - lse[t,h]) v[j]
+        block_lse[t,h,b]  = log sum_{j in J_b(t)} exp(s_j)
+        block_score[t,b]  = sum_h exp(block_lse[t,h,b] - lse[t,h])
+
+    that is, dense causal attention and step 1's outputs from one set of
+    logits.  Blocks after bq(t) get block_lse = -inf and score 0.  Returns
+    dict(out [R,H,Dv], lse [R,H], block_lse [R,H,NBmax], block_score
+    [R,NBmax]) in float64.
+    """
+    q = _f64(q)
+    kf = _f64(k)
+    vf = _f64(v)
+    T, H, Dk = q.shape
+    Dv = vf.shape[1]
+    B = int(block_size)
+    sc = _scale(scale, Dk)
+    bounds = doc_bounds(cu_seqlens)
+    nbmax = max([num_blocks(e - b, B) for b, e in bounds] + [0])
+    doc = _doc_of_rows(cu_seqlens, T)
+    rr = _rows(rows, T)
+    R = rr.shape[0]
+    out = np.empty((R, H, Dv))
+    lse = np.empty((R, H))
+    blse = np.full((R, H, nbmax), -np.inf)
+    score = np.zeros((R, nbmax))
+    for i, t in enumerate(rr):
+        bos, eos = bounds[doc[t]]
+        s = sc * (q[t] @ kf[bos:t + 1].T)                   # [H, n] causal logits
+        m = s.max(axis=1)
+        lse[i] = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+        out[i] = np.exp(s - lse[i][:, None]) @ vf[bos:t + 1]
+        n = t - bos + 1
+        nb = num_blocks(n, B)
+        for b in range(nb):
+            seg = s[:, b * B:min((b + 1) * B, n)]
+            bm = seg.max(axis=1)
+            blse[i, :, b] = bm + np.log(np.exp(seg - bm[:, None]).sum(axis=1))
+        acc = np.zeros(nb)
+        for h in range(H):                                 # increasing head order
+            acc = acc + np.exp(blse[i, h, :nb] - lse[i, h])
+        score[i, :nb] = acc
+    return {"out": out, "lse": lse, "block_lse": blse, "block_score": score}

@@ -381,3 +381,83 @@ def test_sampled_rows_match_full():
     s = O.sparse_mqa_fwd(q, k, v, idx, cu, 8, sink=sink)
     sp = O.sparse_mqa_fwd(q, k, v, idx[rows], cu, 8, sink=sink, rows=rows)
     np.testing.assert_array_equal(sp["out"], s["out"][rows])
+
+
+# ---------------------------------------------------------------------------
+# the full layer's forward with block scores
+# ---------------------------------------------------------------------------
+
+def test_full_layer_matches_torch_sdpa_and_logsumexp():
+    """out against torch float64 causal SDPA document by document; lse and
+    every block's LSE against torch.logsumexp over the masked logits."""
+    docs = [29, 41]
+    q, k, v, _, cu = _inputs(70, 3, 16, 8, docs=docs, seed=31)
+    sc = 0.35
+    f = O.full_layer_fwd(q, k, v, cu, 8, scale=sc)
+    for bos, eos in O.doc_bounds(cu):
+        Q = torch.from_numpy(q[bos:eos]).permute(1, 0, 2)
+        K = torch.from_numpy(k[bos:eos])[None].expand(3, -1, -1)
+        V = torch.from_numpy(v[bos:eos])[None].expand(3, -1, -1)
+        ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, is_causal=True, scale=sc)
+        np.testing.assert_allclose(f["out"][bos:eos], ref.permute(1, 0, 2).numpy(), rtol=1e-12,
+                                   atol=1e-13)
+    logits, _ = _masked_logits(q, k, cu, sc)
+    ref = torch.logsumexp(torch.from_numpy(logits), dim=-1).numpy()
+    np.testing.assert_allclose(f["lse"], ref, rtol=1e-14, atol=1e-14)
+    for t in (0, 7, 8, 28, 29, 37, 69):
+        bos = 0 if t < 29 else 29
+        for b in range((t - bos) // 8 + 1):
+            lo, hi = bos + 8 * b, min(bos + 8 * (b + 1), t + 1)
+            ref_b = torch.logsumexp(torch.from_numpy(logits[t, :, lo:hi]), dim=-1).numpy()
+            np.testing.assert_allclose(f["block_lse"][t, :, b], ref_b, rtol=1e-14)
+
+
+def test_full_layer_block_closed_forms():
+    """Per head the block LSEs log-sum-exp to the row LSE, so the scores sum
+    to H; blocks past the query's own carry -inf / 0."""
+    q, k, v, _, cu = _inputs(90, 5, 8, 4, docs=[7, 33, 50], seed=32)
+    f = O.full_layer_fwd(q, k, v, cu, 16, scale=0.5)
+    lse_b = torch.logsumexp(torch.from_numpy(f["block_lse"]), dim=-1).numpy()
+    np.testing.assert_allclose(lse_b, f["lse"], rtol=1e-13)
+    np.testing.assert_allclose(f["block_score"].sum(axis=1), 5.0, rtol=1e-12)
+    for bos, eos in O.doc_bounds(cu):
+        for t in range(bos, eos):
+            bq = (t - bos) // 16
+            assert np.all(f["block_score"][t, bq + 1:] == 0.0)
+            assert np.all(np.isneginf(f["block_lse"][t, :, bq + 1:]))
+
+
+def test_full_layer_matches_loops():
+    """Brute force: the pure-loop block scorer and the loop attention over
+    an explicit causal mask."""
+    docs = [13, 27]
+    T = sum(docs)
+    q, k, v, _, cu = _inputs(T, 2, 6, 3, docs=docs, seed=33)
+    sc = 0.7
+    f = O.full_layer_fwd(q, k, v, cu, 4, scale=sc)
+    lse, blse, score = loops.block_scores(q.tolist(), k.tolist(), cu, 4, sc)
+    np.testing.assert_allclose(f["lse"], lse, rtol=1e-13)
+    np.testing.assert_allclose(f["block_score"], score, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(f["block_lse"], blse, rtol=1e-13)
+    out, lse2 = loops.masked_attention(q.tolist(), k.tolist(), v.tolist(),
+                                       loops.mask_causal(T, cu), None, sc)
+    np.testing.assert_allclose(f["out"], out, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(f["lse"], lse2, rtol=1e-13)
+
+
+def test_full_layer_rows_and_separate_steps():
+    """Sampled rows equal the full result; the fused definition equals step
+    1 plus dense causal attention without a sink computed separately."""
+    docs = [50, 14, 36]
+    q, k, v, _, cu = _inputs(100, 4, 16, 12, docs=docs, seed=34)
+    f = O.full_layer_fwd(q, k, v, cu, 16)
+    rows = np.array([0, 13, 49, 50, 63, 64, 99])
+    fr = O.full_layer_fwd(q, k, v, cu, 16, rows=rows)
+    for key in ("out", "lse", "block_lse", "block_score"):
+        np.testing.assert_array_equal(fr[key], f[key][rows])
+    bs = O.block_score(q, k, cu, 16)
+    d = O.dense_causal_fwd(q, k, v, cu, sink=None)
+    np.testing.assert_allclose(f["block_score"], bs["block_score"], rtol=1e-13, atol=1e-16)
+    np.testing.assert_array_equal(np.isneginf(f["block_lse"]), np.isneginf(bs["block_lse"]))
+    np.testing.assert_allclose(f["out"], d["out"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(f["lse"], d["lse"], rtol=1e-14)
