@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the (separately timed) backward of the two attention steps")
+    ap.add_argument("--no-full-layer", action="store_true",
+                    help="skip the (separately timed) full layer's fused forward")
     ap.add_argument("--cpu-rows", type=int, default=3072,
                     help="query rows of the oracle sample (cpu_baseline / reference arm)")
     return ap.parse_args()
@@ -125,6 +127,13 @@ def sparse_pairs(idx, cu, B):
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock and clock-event reasons during the timed region.  NVML is
+    read from a background thread every 2 ms (a timed region of a few tens
+    of milliseconds still gets samples); without NVML, nvidia-smi -lms runs
+    as a child process.  start() returns once the first sample is in, so the
+    timed region that follows is covered from its first step."""
+
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -132,47 +141,95 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
+        self.nvml = None
         self.lines = []
+        self.sm = []
+        self.reasons = set()
+        self.smax = None
+        self.source = None
+        self._stop = threading.Event()
 
-    def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+    def _start_nvml(self):
+        import pynvml
+        pynvml.nvmlInit()
+        pr = torch.cuda.get_device_properties(self.dev)
+        bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+        h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+
+        def poll():
+            while not self._stop.is_set():
+                self.sm.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for nm, b in bits.items():
+                    if r & b:
+                        self.reasons.add(nm)
+                time.sleep(0.002)
+
+        self.nvml = pynvml
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
+        self.source = "nvml"
+
+    def _start_smi(self):
+        self.proc = subprocess.Popen(
+            ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+             "--format=csv,noheader,nounits", "-lms", "20"],
+            stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        self.source = "nvidia-smi"
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
+            parts = [p.strip() for p in line.strip().split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
+                sm, smax = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for nm, val in zip(names, parts[5:9]):
+            if self._stop.is_set():
+                break
+            self.sm.append(sm)
+            self.smax = smax
+            for nm, val in zip(self.NAMES, parts[5:9]):
                 if val.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                    self.reasons.add(nm)
+
+    def start(self):
+        try:
+            self._start_nvml()
+        except Exception:
+            try:
+                self._start_smi()
+            except (OSError, FileNotFoundError):
+                self.proc = None
+                return
+        t0 = time.time()
+        while not self.sm and time.time() - t0 < 5.0:
+            time.sleep(0.001)
+        self.sm.clear()  # keep only samples taken from here on
+        self.reasons.clear()
+
+    def stop(self):
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock source unavailable"]}
+        self._stop.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.thread.join(timeout=5)
+        sm = list(self.sm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
+                "reasons": sorted(self.reasons), "samples": len(sm), "source": self.source}
 
 
 # ---------------------------------------------------------------------------
@@ -402,6 +459,9 @@ def run_ours(args, wl, world, rank):
     bwd = None
     if not args.no_backward:
         bwd = run_backward(inp, wl, step, cu, pk)
+    full = None
+    if not args.no_full_layer:
+        full = run_full_layer(inp, wl, pk, flush, avg["score"])
 
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -421,8 +481,54 @@ def run_ours(args, wl, world, rank):
         "clocks": clk,
         "e2e": e2e,
         "backward": bwd,
+        "full_layer": full,
     }
     return res
+
+
+def run_full_layer(inp, wl, pk, flush, score_ms, reps=3):
+    """The full layer's forward with step 1 fused in (not part of the
+    headline step, which uses step 1 alone): CUDA-event time per call with L2
+    flushed before each, one untimed call first.  Algorithmic work per causal
+    (query, key) pair and head: 2 Dk (scores) + 2 Dv (PV) flops."""
+    T, H = wl.total_tokens, wl.num_heads
+    dev = inp.q.device
+    nb = hs.nbmax(inp.max_seqlen, wl.block_size)
+    out = torch.empty((T, H, wl.dv), device=dev, dtype=inp.q.dtype)
+    lse = torch.empty((T, H), device=dev, dtype=torch.float32)
+    bs = torch.empty((T, nb), device=dev, dtype=torch.float32)
+    ws = torch.empty(max(1, hs.workspace_size(hs.HS_OP_BLOCK_SCORE_ATTN, T, len(wl.docs()),
+                                              inp.max_seqlen, H, wl.dk, wl.dv, wl.dtype,
+                                              wl.block_size)), device=dev, dtype=torch.uint8)
+
+    def fn():
+        hs.hs_block_score_attn_fwd(inp.q, inp.k, inp.v, inp.cu_seqlens, inp.max_seqlen,
+                                   wl.block_size, out=out, lse=lse, out_block_score=bs,
+                                   workspace=ws)
+
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for r in range(reps):
+        flush.fill_(r & 0xff)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    hs.poll_status(dev)
+    ms = statistics.mean(ts)
+    fl = 2.0 * H * (wl.dk + wl.dv) * causal_pairs(wl.docs())
+    tf = fl / (ms / 1e3) / 1e12
+    return {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / pk["bf16_tflops"],
+            "frac_of_nominal_bf16": tf / NOMINAL_BF16_TFLOPS, "algorithmic_flops": fl,
+            "calls_timed": reps, "block_score_step_ms": score_ms,
+            "tokens_per_s": T / (ms / 1e3),
+            "path": "tcgen05" if hs.path(hs.HS_OP_BLOCK_SCORE_ATTN, wl.dtype, H, wl.dk, wl.dv,
+                                         wl.block_size) == hs.HS_PATH_TCGEN05 else "simt",
+            "outputs": "out, lse, block_score (dense causal attention + step 1, no sink)"}
 
 
 def run_backward(inp, wl, step, cu, pk, reps=2):

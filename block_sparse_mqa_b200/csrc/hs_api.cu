@@ -170,6 +170,7 @@ int hs_path(int op, hs_dtype dtype, int num_heads, int dk, int dv, int block_siz
       return HS_PATH_SIMT;
     case HS_OP_SPARSE_MQA:
     case HS_OP_SWA_MQA:
+    case HS_OP_BLOCK_SCORE_ATTN:  // fused, or the attention then the score kernel
       if (dtype == HS_BF16 && !g_force_simt.load() &&
           hs::tc_attention_supported(num_heads, dk, dv, block_size, op == HS_OP_SPARSE_MQA))
         return HS_PATH_TCGEN05;
@@ -184,12 +185,22 @@ size_t hs_workspace_size(int op, int total_tokens, int num_docs, int max_seqlen,
   if ((op == HS_OP_SPARSE_MQA_BWD || op == HS_OP_SWA_MQA_BWD) && total_tokens > 0 &&
       num_heads > 0)
     return hs::simt_backward_workspace(total_tokens, num_heads);
-  if (op != HS_OP_BLOCK_SCORE || total_tokens <= 0 || !valid_block(block_size)) return 0;
+  if ((op != HS_OP_BLOCK_SCORE && op != HS_OP_BLOCK_SCORE_ATTN) || total_tokens <= 0 ||
+      !valid_block(block_size))
+    return 0;
   const int nbmax = nbmax_of(max_seqlen, block_size);
+  size_t need = 0;
   if (dtype == HS_BF16 && !g_force_simt.load() &&
       hs::tc_block_score_supported(num_heads, dk, block_size, nbmax))
-    return hs::tc_block_score_workspace(total_tokens, num_docs, num_heads, nbmax);
-  return 0;
+    need = hs::tc_block_score_workspace(total_tokens, num_docs, num_heads, nbmax);
+  // the fused kernel's scratch (the call falls back to the score kernel when
+  // pointer alignment rules the fused one out, so cover both)
+  if (op == HS_OP_BLOCK_SCORE_ATTN && dtype == HS_BF16 && !g_force_simt.load() &&
+      hs::tc_full_supported(num_heads, dk, dv, block_size)) {
+    const size_t f = hs::tc_full_workspace(total_tokens, nbmax);
+    if (f > need) need = f;
+  }
+  return need;
 }
 
 hs_status hs_poll_status(hs_stream_t stream) {
@@ -346,6 +357,74 @@ hs_status hs_swa_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_str
   return attention_common(a, false, q, q_row_stride, q_head_stride, k, k_row_stride, v,
                           v_row_stride, cu_seqlens, num_docs, total_tokens, max_seqlen,
                           num_heads, dk, dv, dtype, softmax_scale, sink, out, lse, stream);
+}
+
+hs_status hs_block_score_attn_fwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                                  const void* k, int64_t k_row_stride, const void* v,
+                                  int64_t v_row_stride, const int32_t* cu_seqlens, int num_docs,
+                                  int total_tokens, int max_seqlen, int num_heads, int dk, int dv,
+                                  hs_dtype dtype, float softmax_scale, int block_size, void* out,
+                                  float* lse, float* block_score, int nb_stride, float* block_lse,
+                                  void* workspace, size_t workspace_bytes, hs_stream_t stream) {
+  hs::FullArgs f{};
+  hs_status r = check_problem(f.p, q, q_row_stride, q_head_stride, k, k_row_stride, cu_seqlens,
+                              num_docs, total_tokens, max_seqlen, num_heads, dk, dv, dtype,
+                              softmax_scale);
+  if (r != HS_OK) return r;
+  if (!valid_block(block_size))
+    return fail(HS_ERR_UNSUPPORTED, "block_size %d not in {16, 32, 64, 128}", block_size);
+  if (dv < 1) return fail(HS_ERR_UNSUPPORTED, "dv must be >= 1");
+  if (!v) return fail(HS_ERR_INVALID_ARG, "v is NULL");
+  if (v_row_stride < dv) return fail(HS_ERR_INVALID_ARG, "v_row_stride %lld < dv",
+                                     (long long)v_row_stride);
+  if (!out || !lse || !block_score) return fail(HS_ERR_INVALID_ARG, "out, lse or block_score is NULL");
+  if (total_tokens == 0) return HS_OK;
+  const int nbmax = nbmax_of(max_seqlen, block_size);
+  if (nb_stride < nbmax)
+    return fail(HS_ERR_INVALID_ARG, "nb_stride %d < ceil(max_seqlen / block_size) = %d", nb_stride,
+                nbmax);
+  f.p.v = v;
+  f.p.v_row_stride = v_row_stride;
+  f.block_size = block_size;
+  f.nbmax = nbmax;
+  f.nb_stride = nb_stride;
+  f.out = out;
+  f.lse = lse;
+  f.block_score = block_score;
+  f.block_lse = block_lse;
+  f.workspace = workspace;
+  r = status_ptr(&f.p.status);
+  if (r != HS_OK) return r;
+  hs::AttnArgs a{};  // the attention part, for the eligibility test and the two-kernel path
+  a.p = f.p;
+  a.block_size = block_size;
+  a.window = max_seqlen;  // covers every document: dense causal
+  a.sink = nullptr;
+  a.out = out;
+  a.lse = lse;
+  const bool fused = dtype == HS_BF16 && !g_force_simt.load() &&
+                     hs::tc_full_supported(num_heads, dk, dv, block_size) &&
+                     hs::tc_attention_eligible(a);
+  if (fused) {
+    const size_t need = hs::tc_full_workspace(total_tokens, nbmax);
+    if (!workspace || workspace_bytes < need)
+      return fail(HS_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                  workspace ? workspace_bytes : (size_t)0);
+    return launched(hs::launch_tc_full(f, g_wait_limit.load(), stream), "tc full layer");
+  }
+  // two kernels: the attention (its lse is the same quantity; the score
+  // kernel then writes lse again), then step 1
+  const bool tca = dtype == HS_BF16 && !g_force_simt.load() &&
+                   hs::tc_attention_supported(num_heads, dk, dv, block_size, false) &&
+                   hs::tc_attention_eligible(a);
+  r = launched(tca ? hs::launch_tc_attention(a, false, g_wait_limit.load(), stream)
+                   : hs::launch_simt_attention(a, false, stream),
+               "full layer attention");
+  if (r != HS_OK) return r;
+  return hs_block_score(q, q_row_stride, q_head_stride, k, k_row_stride, cu_seqlens, num_docs,
+                        total_tokens, max_seqlen, num_heads, dk, dtype, softmax_scale,
+                        block_size, lse, block_score, nb_stride, block_lse, workspace,
+                        workspace_bytes, stream);
 }
 
 static hs_status backward_common(hs::BwdArgs& a, bool sparse, const void* q, int64_t qrs,

@@ -44,6 +44,18 @@ struct AttnArgs {
   float* lse;
 };
 
+// The full layer's fused forward (after host validation): dense causal
+// attention without a sink plus step 1's outputs.
+struct FullArgs {
+  Problem p;
+  int block_size, nbmax, nb_stride;
+  void* out;
+  float* lse;
+  float* block_score;
+  float* block_lse;  // may be null
+  void* workspace;   // tc_full_workspace() bytes on the tensor-core path
+};
+
 // Backward of the attention calls (after host validation).
 struct BwdArgs {
   Problem p;
@@ -89,6 +101,10 @@ bool tc_attention_supported(int num_heads, int dk, int dv, int block_size, bool 
 bool tc_attention_eligible(const AttnArgs& a);  // alignment conditions
 cudaError_t launch_tc_attention(const AttnArgs& a, bool sparse, long long wait_limit,
                                 cudaStream_t s);
+// Full-layer mode of the same kernel (block sizes 32, 64, 128).
+bool tc_full_supported(int num_heads, int dk, int dv, int block_size);
+size_t tc_full_workspace(int total_tokens, int nbmax);
+cudaError_t launch_tc_full(const FullArgs& f, long long wait_limit, cudaStream_t s);
 
 // Records msg as the calling thread's hs_last_error() and returns st.
 hs_status report_error(hs_status st, const char* msg);

@@ -1,5 +1,6 @@
-// hs_sparse_mqa_fwd and hs_swa_mqa_fwd on tcgen05 tensor cores (bf16 in,
-// fp32 accumulate), 64 query heads over one KV head.
+// hs_sparse_mqa_fwd, hs_swa_mqa_fwd and the full layer's fused forward
+// (hs_block_score_attn_fwd) on tcgen05 tensor cores (bf16 in, fp32
+// accumulate), 64 query heads over one KV head.
 //
 // Definitions ("HySparse MQA sparse attention ...", PaddleFleet pull request
 // 1470, "Core" list: block-sparse DSA gather and SWA sliding-window MQA, both
@@ -8,6 +9,11 @@
 //   lse[t,h] = log(exp(sink_h) + sum_{j in S_t} exp(s_j)),
 //   out[t,h] = sum_{j in S_t} exp(s_j - lse[t,h]) v_j,
 // with S_t the selected blocks (causal inside the own block) or the window.
+// The full layer ("Core" list: FA4-fused block scoring; the Copilot overview:
+// the HySparse full layer yields the block indices) attends every causal key
+// without a sink and also emits, from the same fp32 exponentials,
+//   block_lse[t,h,b] = log sum_{j in block b, j <= t} exp(s_j),
+//   block_score[t,b] = sum_h exp(block_lse[t,h,b] - lse[t,h]).
 //
 // Design.  Every query token has its own key set, so its 64 heads are the
 // only rows that share a key tile.  The kernel therefore works transposed:
@@ -32,6 +38,18 @@
 // owner, warp 11 = PV issuer, warps 2-9 = two softmax warpgroups, each
 // owning 32 of the 64 heads (per-head state never crosses warpgroups).  All
 // waits are bounded (HS_ERR_TIMEOUT, drain, free).
+//
+// Full-layer mode: each key tile covers 128 / B whole blocks (B >= 32, so a
+// block is one or more whole warps of key rows).  After the exponentials
+// every warp transposes-and-sums its 32 rows per head; at the warpgroup's
+// next rendezvous the warps of each block add their sums and write
+// log2(sum) + running max (the block's LSE in log2 units) to a per-CTA
+// scratch row [block][head] in global memory (L2-resident; two rows per CTA,
+// alternating by token, since one token's rows are read while the next
+// token's are written).  After the token's last tile both warpgroups meet
+// (a bounded 256-thread barrier) and each warp turns blocks into scores:
+// lanes take two heads each, exp2(block LSE - row LSE), a fixed-order warp
+// sum.
 
 #include <math.h>
 
@@ -61,6 +79,8 @@ constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kRescaleLog2 = 8.f;  // raise the running max only past 2^8
 
+constexpr int kModeSwa = 0, kModeSparse = 1, kModeFull = 2;
+
 struct AttnParams {
   const int32_t* cu;
   int num_docs, T, max_seqlen;
@@ -74,6 +94,11 @@ struct AttnParams {
   float* lse;
   int* status;
   long long wait_ns;
+  // full-layer mode only
+  float* blk;          // scratch: [gridDim.x][2][nbmax][kH] block LSEs (log2 units)
+  int nbmax, nb_stride;
+  float* block_score;  // [T, nb_stride]
+  float* block_lse;    // [T, kH, nb_stride] or null
 };
 
 struct Shared {
@@ -83,7 +108,10 @@ struct Shared {
   uint64_t sfull[2], sempty[2];
   uint64_t pfull, pvdone, ofull, oempty, drain, drain_pv;
   uint64_t rv[2];            // rendezvous inside softmax warpgroup wg (128 threads)
+  uint64_t rv_all;           // rendezvous of both softmax warpgroups (full-layer mode)
   float red[2][4][32];       // [warpgroup][warp][lane] partial reductions
+  float bsum[2][4][32];      // [warpgroup][warp][head] one tile's exp sums (full layer)
+  float lse2[kH];            // row LSE per head, log2 units (full layer)
   float mrun[kH];            // running max per head (log2 domain)
   float alpha[kH];           // rescale factor per head
   float lsum[kH];            // output multiplier per head
@@ -219,11 +247,13 @@ __device__ __forceinline__ void pv_run(uint32_t d, uint64_t a0, uint64_t b0, uin
             (FIRST && kk == 0) ? 0u : 1u);
 }
 
-template <bool kSparse>
+template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap,
                     const __grid_constant__ CUtensorMap qmap, const AttnParams p) {
+  constexpr bool kSparse = kMode == kModeSparse;
+  constexpr bool kFull = kMode == kModeFull;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -250,6 +280,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       mbar_init(&sh->sempty[b], 256);
       mbar_init(&sh->rv[b], 128);
     }
+    mbar_init(&sh->rv_all, 256);
     mbar_init(&sh->pfull, 256);
     mbar_init(&sh->pvdone, 1);
     mbar_init(&sh->ofull, 1);
@@ -480,11 +511,28 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
     const uint32_t lane_base = tmem + ((uint32_t)(32 * g4) << 16);
     const float sl2 = p.scale_log2;
     const int dvs = p.dv;  // row stride of out
-    uint32_t sidx = 0, npv = 0, rvph = 0, ntok = 0, gt = 0;
+    uint32_t sidx = 0, npv = 0, rvph = 0, ntok = 0, gt = 0, rvph_all = 0;
     bool ok = true;
+    // full layer: blocks per tile, warps per block, the running max (log2)
+    // of this lane's head that the last tile's exponentials used
+    const int nbt = kFull ? kTile / p.B : 0;
+    const int wpb = kFull ? p.B / 32 : 1;
+    float m_used = 0.f;
     for (int t = blockIdx.x; t < p.T && ok && !aborted(sh); t += G) {
       const TokenPlan tp = plan_token<kSparse>(p, t, false);
       if (!tp.ok) continue;
+      float* const blkrow =
+          kFull ? p.blk + ((size_t)blockIdx.x * 2 + (ntok & 1)) * (size_t)p.nbmax * kH : nullptr;
+      // block LSEs (log2 units) of tile `tile`: the warps of each block add
+      // their per-head sums; blocks past the query's own are not stored
+      auto flush_blocks = [&](int tile) {
+        if (g4 < nbt) {
+          float sum = 0.f;
+          for (int w = 0; w < wpb; ++w) sum += sh->bsum[wg][g4 * wpb + w][lane];
+          const int b = tile * nbt + g4;
+          if (b <= tp.bq) blkrow[(size_t)b * kH + hb + lane] = m_used + fast_log2(sum);
+        }
+      };
       if (tp.ntile == 0) {  // no valid block: empty softmax, only the sink
         for (int e = r; e < 32 * dvs; e += 128)
           p.out[((int64_t)t * kH + hb) * dvs + e] = __float2bfloat16_rn(0.f);
@@ -541,6 +589,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           sh->red[wg][g4][lane] = tr_max(a);
         }
         if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
+        if (kFull && i > 0) flush_blocks(i - 1);  // sums written before this rendezvous
         if (g4 == 0) {
           const int hh = hb + lane;
           const float tm = fmaxf(fmaxf(sh->red[wg][0][lane], sh->red[wg][1][lane]),
@@ -573,6 +622,14 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           lpart[2 * k + 1] += e1;
           __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
           pk[k] = *reinterpret_cast<uint32_t*>(&pr);
+          if (kFull) {
+            x[2 * k] = e0;
+            x[2 * k + 1] = e1;
+          }
+        }
+        if (kFull) {  // this warp's 32 key rows summed per head (lane = head)
+          sh->bsum[wg][g4][lane] = tr_sum(x);
+          m_used = sh->mrun[hb + lane];
         }
         // P^T may be rewritten once PV of the previous tile has read it
         if (i > 0) {
@@ -611,6 +668,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       // ---------------- epilogue: per-head sums, sink, normalisation
       sh->red[wg][g4][lane] = tr_sum(lpart);
       if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
+      if (kFull) flush_blocks(tp.ntile - 1);
       if (g4 == 0) {
         const int hh = hb + lane;
         const float l = (sh->red[wg][0][lane] + sh->red[wg][1][lane]) +
@@ -620,7 +678,8 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         const float M = fmaxf(m, sk);
         const float den = l * fast_exp2(m - M) + fast_exp2(sk - M);
         sh->lsum[hh] = fast_exp2(m - M) / den;
-        p.lse[(int64_t)t * kH + hh] = (M + fast_log2(den)) * kLn2;
+        sh->lse2[hh] = M + fast_log2(den);
+        p.lse[(int64_t)t * kH + hh] = sh->lse2[hh] * kLn2;
       }
       // the last PV of this token must be complete before O^T is read
       if (!mbar_wait(&sh->pvdone, npv & 1, lim)) { ok = false; break; }
@@ -661,6 +720,32 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       }
       tc_fence_before();
       mbar_arrive(&sh->oempty);
+      if (kFull) {
+        // both warpgroups' block LSEs and row LSEs are in place after this
+        __threadfence_block();
+        mbar_arrive(&sh->rv_all);
+        if (!mbar_wait(&sh->rv_all, rvph_all, lim)) { ok = false; break; }
+        rvph_all ^= 1;
+        const float la = sh->lse2[lane], lb = sh->lse2[lane + 32];
+        float* const srow = p.block_score + (int64_t)t * p.nb_stride;
+        float* const lrow = p.block_lse ? p.block_lse + (int64_t)t * kH * p.nb_stride : nullptr;
+        for (int b = wg * 4 + g4; b < p.nbmax; b += 8) {  // one block per warp
+          float sc = 0.f, va = -INFINITY, vb = -INFINITY;
+          if (b <= tp.bq) {
+            va = __ldcg(blkrow + (size_t)b * kH + lane);
+            vb = __ldcg(blkrow + (size_t)b * kH + lane + 32);
+            float e = fast_exp2(va - la) + fast_exp2(vb - lb);
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) e += __shfl_xor_sync(0xffffffffu, e, off);
+            sc = e;
+          }
+          if (lane == 0) srow[b] = sc;
+          if (lrow) {
+            lrow[(int64_t)lane * p.nb_stride + b] = va * kLn2;
+            lrow[(int64_t)(lane + 32) * p.nb_stride + b] = vb * kLn2;
+          }
+        }
+      }
       ++ntok;
       // lsum / mrun / blist are rewritten for the next token only after this
       if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
@@ -690,8 +775,11 @@ bool tc_attention_eligible(const AttnArgs& a) {
          p.q_head_stride % 8 == 0 && p.k_row_stride % 8 == 0 && p.v_row_stride % 8 == 0;
 }
 
-cudaError_t launch_tc_attention(const AttnArgs& a, bool sparse, long long wait_limit,
-                                cudaStream_t s) {
+namespace {
+
+cudaError_t launch_mode(const AttnArgs& a, int mode, const FullArgs* fa, long long wait_limit,
+                        cudaStream_t s) {
+  const bool sparse = mode == kModeSparse;
   const Problem& p = a.p;
   const uint32_t rows = sparse ? (uint32_t)a.block_size : (uint32_t)kTile;
   CUtensorMap kmap, vmap, qmap;
@@ -721,7 +809,7 @@ cudaError_t launch_tc_attention(const AttnArgs& a, bool sparse, long long wait_l
   ap.idx = a.idx;
   ap.topk = a.topk;
   ap.B = a.block_size;
-  ap.window = a.window;
+  ap.window = mode == kModeFull ? (1 << 30) : a.window;  // full layer: every causal key
   ap.nck = p.dk / 64;
   ap.nvc = (p.dv + 127) / 128;  // a panel past Dv is zero-filled by TMA
   ap.dv = p.dv;
@@ -731,13 +819,49 @@ cudaError_t launch_tc_attention(const AttnArgs& a, bool sparse, long long wait_l
   ap.lse = a.lse;
   ap.status = p.status;
   ap.wait_ns = wait_limit > 0 ? wait_limit : kDefaultWaitNs;
+  ap.blk = fa ? static_cast<float*>(fa->workspace) : nullptr;
+  ap.nbmax = fa ? fa->nbmax : 0;
+  ap.nb_stride = fa ? fa->nb_stride : 0;
+  ap.block_score = fa ? fa->block_score : nullptr;
+  ap.block_lse = fa ? fa->block_lse : nullptr;
   const int grid = p.total_tokens < sm_count() ? p.total_tokens : sm_count();
-  auto kern = sparse ? tc_attention_kernel<true> : tc_attention_kernel<false>;
+  auto kern = mode == kModeSparse ? tc_attention_kernel<kModeSparse>
+              : mode == kModeFull ? tc_attention_kernel<kModeFull>
+                                  : tc_attention_kernel<kModeSwa>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, s>>>(kmap, vmap, qmap, ap);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc_attention(const AttnArgs& a, bool sparse, long long wait_limit,
+                                cudaStream_t s) {
+  return launch_mode(a, sparse ? kModeSparse : kModeSwa, nullptr, wait_limit, s);
+}
+
+bool tc_full_supported(int num_heads, int dk, int dv, int block_size) {
+  return tc_attention_supported(num_heads, dk, dv, block_size, false) && block_size >= 32;
+}
+
+size_t tc_full_workspace(int total_tokens, int nbmax) {
+  const int grid = total_tokens < sm_count() ? total_tokens : sm_count();
+  return (size_t)grid * 2 * (size_t)nbmax * kH * sizeof(float);
+}
+
+cudaError_t launch_tc_full(const FullArgs& f, long long wait_limit, cudaStream_t s) {
+  AttnArgs a{};
+  a.p = f.p;
+  a.idx = nullptr;
+  a.topk = 0;
+  a.block_size = f.block_size;
+  a.window = 0;
+  a.sink = nullptr;
+  a.out = f.out;
+  a.lse = f.lse;
+  return launch_mode(a, kModeFull, &f, wait_limit, s);
 }
 
 }  // namespace hs

@@ -37,6 +37,7 @@ HS_OP_SPARSE_MQA = 2
 HS_OP_SWA_MQA = 3
 HS_OP_SPARSE_MQA_BWD = 4
 HS_OP_SWA_MQA_BWD = 5
+HS_OP_BLOCK_SCORE_ATTN = 6
 
 HS_PATH_SIMT = 0
 HS_PATH_TCGEN05 = 1
@@ -48,6 +49,7 @@ EXPORTS = (
     "hs_workspace_size", "hs_path", "hs_poll_status", "hs_set_force_simt",
     "hs_selftest_wait", "hs_status_string", "hs_last_error", "hs_version",
     "hs_block_score_static", "hs_sparse_mqa_bwd", "hs_swa_mqa_bwd",
+    "hs_block_score_attn_fwd",
 )
 
 
@@ -90,6 +92,9 @@ def lib() -> ctypes.CDLL:
     L.hs_swa_mqa_bwd.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _int, _int, _int,
                                  _int, _int, _int, _int, _flt, _int, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _vp, _vp, _vp, _szt, _vp]
+    L.hs_block_score_attn_fwd.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _int, _int,
+                                          _int, _int, _int, _int, _int, _flt, _int, _vp, _vp,
+                                          _vp, _int, _vp, _vp, _szt, _vp]
     L.hs_workspace_size.argtypes = [_int] * 9
     L.hs_workspace_size.restype = _szt
     L.hs_path.argtypes = [_int] * 6
@@ -104,7 +109,7 @@ def lib() -> ctypes.CDLL:
     L.hs_last_error.restype = ctypes.c_char_p
     for fn in ("hs_block_score", "hs_select_topk", "hs_sparse_mqa_fwd", "hs_swa_mqa_fwd",
                "hs_poll_status", "hs_block_score_static", "hs_sparse_mqa_bwd",
-               "hs_swa_mqa_bwd"):
+               "hs_swa_mqa_bwd", "hs_block_score_attn_fwd"):
         getattr(L, fn).restype = _int
     _lib = L
     return L
@@ -182,6 +187,20 @@ def nbmax(max_seqlen: int, block_size: int) -> int:
     return (max_seqlen + block_size - 1) // block_size
 
 
+def _check_block_outputs(bs, blse, T, H, nb):
+    """block_score [T, nb_stride] and block_lse [T, H, nb_stride] share one
+    column stride (nb_stride >= NBmax) in the C calls."""
+    if bs.dtype != torch.float32 or bs.dim() != 2 or bs.shape[0] != T or bs.stride(1) != 1 \
+            or bs.stride(0) < nb or bs.shape[1] < nb:
+        raise ValueError("block_score must be float32 [T, >= NBmax] with contiguous rows")
+    if blse is not None:
+        ns = bs.stride(0)
+        if blse.dtype != torch.float32 or tuple(blse.shape) != (T, H, ns) or \
+                not blse.is_contiguous():
+            raise ValueError("block_lse must be contiguous float32 [T, H, nb_stride] with the "
+                             "block_score row stride")
+
+
 def hs_block_score(q, k, cu_seqlens, max_seqlen: int, block_size: int,
                    softmax_scale: float = 0.0, want_block_lse: bool = False,
                    out_lse=None, out_block_score=None, out_block_lse=None, workspace=None):
@@ -198,6 +217,7 @@ def hs_block_score(q, k, cu_seqlens, max_seqlen: int, block_size: int,
     blse = out_block_lse
     if want_block_lse and blse is None:
         blse = torch.empty((T, H, nb), device=dev, dtype=f32)
+    _check_block_outputs(bs, blse, T, H, nb)
     nd = cu_seqlens.numel() - 1
     need = workspace_size(HS_OP_BLOCK_SCORE, T, nd, max_seqlen, H, Dk, 0, q.dtype, block_size)
     if workspace is None and need > 0:
@@ -289,6 +309,41 @@ def hs_swa_mqa_fwd(q, k, v, cu_seqlens, max_seqlen: int, window: int, sink=None,
         cu_seqlens.numel() - 1, T, int(max_seqlen), H, Dk, v.shape[1], _dtype_code(q),
         float(softmax_scale), int(window), _ptr(sink), _ptr(o), _ptr(l), _stream(q.device)))
     return o, l
+
+
+def hs_block_score_attn_fwd(q, k, v, cu_seqlens, max_seqlen: int, block_size: int,
+                            softmax_scale: float = 0.0, want_block_lse: bool = False, out=None,
+                            lse=None, out_block_score=None, out_block_lse=None, workspace=None):
+    """The full layer's forward with step 1 fused in: dense causal attention
+    (no sink) plus step 1's outputs.  Returns (out [T,H,Dv] in q's dtype,
+    lse [T,H] f32, block_score [T,NBmax] f32, block_lse [T,H,NBmax] f32 or
+    None)."""
+    _need_cuda(q, k, v, cu_seqlens)
+    qrs, qhs, krs = _qk_strides(q, k)
+    if v.dim() != 2 or v.stride(1) != 1:
+        raise ValueError("v must be [T, Dv] with contiguous rows")
+    T, H, Dk = q.shape
+    Dv = v.shape[1]
+    o, l = _attn_out(q, v, out, lse)
+    nb = nbmax(max_seqlen, block_size)
+    dev = q.device
+    bs = out_block_score if out_block_score is not None else torch.empty(
+        (T, nb), device=dev, dtype=torch.float32)
+    blse = out_block_lse
+    if want_block_lse and blse is None:
+        blse = torch.empty((T, H, nb), device=dev, dtype=torch.float32)
+    _check_block_outputs(bs, blse, T, H, nb)
+    nd = cu_seqlens.numel() - 1
+    need = workspace_size(HS_OP_BLOCK_SCORE_ATTN, T, nd, max_seqlen, H, Dk, Dv, q.dtype,
+                          block_size)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    _check(lib().hs_block_score_attn_fwd(
+        _ptr(q), qrs, qhs, _ptr(k), krs, _ptr(v), v.stride(0), _ptr(cu_seqlens), nd, T,
+        int(max_seqlen), H, Dk, Dv, _dtype_code(q), float(softmax_scale), int(block_size),
+        _ptr(o), _ptr(l), _ptr(bs), bs.stride(0), _ptr(blse), _ptr(workspace),
+        0 if workspace is None else workspace.numel(), _stream(dev)))
+    return o, l, bs, blse
 
 
 def _bwd_prep(q, k, v, out, lse, dout, cu_seqlens, sink, op, max_seqlen, grads, workspace):

@@ -18,6 +18,10 @@
  *   hs_sparse_mqa_bwd  dq, dk, dv and the sink gradient of hs_sparse_mqa_fwd
  *   hs_swa_mqa_bwd     the same for hs_swa_mqa_fwd
  *
+ * hs_block_score_attn_fwd is the full layer's forward: dense causal
+ * attention that emits step 1's outputs from the same pass, replacing
+ * hs_block_score where the model runs that layer anyway.
+ *
  * Conventions shared by every call
  * --------------------------------
  * Pointers named q, k, v, out, lse, block_score, block_lse, idx, sink and
@@ -94,7 +98,8 @@ typedef enum hs_op {
   HS_OP_SPARSE_MQA = 2,
   HS_OP_SWA_MQA = 3,
   HS_OP_SPARSE_MQA_BWD = 4,
-  HS_OP_SWA_MQA_BWD = 5
+  HS_OP_SWA_MQA_BWD = 5,
+  HS_OP_BLOCK_SCORE_ATTN = 6
 } hs_op;
 
 /* Kernel family a call will use, as returned by hs_path(). */
@@ -278,6 +283,51 @@ hs_status hs_swa_mqa_bwd(const void* q, int64_t q_row_stride, int64_t q_head_str
                          void* workspace, size_t workspace_bytes, hs_stream_t stream);
 
 /*
+ * The full layer's forward with step 1 fused in.
+ * Source: pull request 1470, "Core" list (FA4-fused block scoring), the
+ * Copilot overview (the HySparse full layer produces the shared KV and the
+ * block indices) and per-file table (block_score_fa4.py: the full layer's
+ * flash-attention forward emits the scaled block_logit; pipeline.py: the
+ * score is recovered as exp(block_logit - lse)); review of pull request 1453
+ * (the PyLayer saves out and lse; per-document block_bos).
+ *
+ * For query t in document [bos, eos), head h, s_j = scale * <q[t,h], k[j]>
+ * over every causal key j in [bos, t], with no sink:
+ *   lse[t,h]          = log sum_j exp(s_j)
+ *   out[t,h]          = sum_j exp(s_j - lse[t,h]) * v[j]
+ *   block_lse[t,h,b]  = log sum_{j in block b, j <= t} exp(s_j)
+ *   block_score[t,b]  = sum_h exp(block_lse[t,h,b] - lse[t,h])
+ * lse, block_score and block_lse are exactly what hs_block_score defines
+ * (blocks past bq(t) up to NBmax: score 0, block_lse -inf; columns NBmax ..
+ * nb_stride-1 not written); out is hs_swa_mqa_fwd's output for a window
+ * covering every document without a sink.
+ *
+ *   out          [T, H, Dv] of `dtype`, contiguous, output.
+ *   lse          [T, H] fp32, output.
+ *   block_score  [T, nb_stride] fp32, output; nb_stride >= NBmax.
+ *   block_lse    [T, H, nb_stride] fp32, optional output (NULL = skip).
+ *   workspace    device scratch of at least hs_workspace_size(
+ *                HS_OP_BLOCK_SCORE_ATTN, ...) bytes; contents on entry do
+ *                not matter; concurrent calls must not share one.  A missing
+ *                or short workspace is HS_ERR_WORKSPACE before any launch.
+ *   block_size   16, 32, 64 or 128.
+ * bf16 with 64 heads, Dk and Dv multiples of 64 (Dk <= 576, Dv <= 512),
+ * block sizes 32..128 and 16-byte aligned q, k, v, out run as ONE tcgen05
+ * kernel (its scratch: two [NBmax, H] fp32 rows per SM).  Other inputs run
+ * the attention and hs_block_score's kernel one after the other on the same
+ * stream (same results, two passes over the logits).
+ */
+hs_status hs_block_score_attn_fwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                                  const void* k, int64_t k_row_stride,
+                                  const void* v, int64_t v_row_stride,
+                                  const int32_t* cu_seqlens, int num_docs, int total_tokens,
+                                  int max_seqlen, int num_heads, int dk, int dv,
+                                  hs_dtype dtype, float softmax_scale, int block_size,
+                                  void* out, float* lse, float* block_score, int nb_stride,
+                                  float* block_lse, void* workspace, size_t workspace_bytes,
+                                  hs_stream_t stream);
+
+/*
  * Step 1 for callers that cannot allocate device memory.
  * The method has no counterpart of this call; it is a deployment aid.
  *
@@ -315,7 +365,8 @@ hs_status hs_block_score_static(const void* q, int64_t q_row_stride, int64_t q_h
 /* ---------------------------------------------------------------- helpers */
 
 /* Bytes of `workspace` that op needs for these sizes (0 = none).
- * HS_OP_BLOCK_SCORE and the two backward ops use a workspace. */
+ * HS_OP_BLOCK_SCORE, HS_OP_BLOCK_SCORE_ATTN and the two backward ops use a
+ * workspace. */
 size_t hs_workspace_size(int op, int total_tokens, int num_docs, int max_seqlen,
                          int num_heads, int dk, int dv, hs_dtype dtype, int block_size);
 

@@ -158,3 +158,30 @@ def test_selftest_rejects_bad_limit():
     L = hs.lib()
     assert L.hs_selftest_wait(0, None) == hs.HS_ERR_INVALID_ARG
     assert L.hs_selftest_wait(10**10, None) == hs.HS_ERR_INVALID_ARG
+
+
+def test_full_layer_rejects_bad_arguments():
+    L = hs.lib()
+    p = ctypes.c_void_p(256)
+    T, H = 100, 64
+    ws = L.hs_workspace_size(hs.HS_OP_BLOCK_SCORE_ATTN, T, 1, 100, H, 576, 512, hs.HS_BF16, 64)
+    # covers the fused kernel's scratch (2 rows of [NBmax, H] fp32 per CTA)
+    # and step 1's kernel, which runs when the fused one is not eligible
+    assert ws >= min(T, 148) * 2 * 2 * H * 4
+    assert ws == L.hs_workspace_size(hs.HS_OP_BLOCK_SCORE, T, 1, 100, H, 576, 0, hs.HS_BF16, 64)
+    assert L.hs_workspace_size(hs.HS_OP_BLOCK_SCORE_ATTN, T, 1, 100, 4, 64, 48, hs.HS_F32, 16) == 0
+    assert L.hs_path(hs.HS_OP_BLOCK_SCORE_ATTN, hs.HS_BF16, H, 576, 512, 64) == hs.HS_PATH_TCGEN05
+    assert L.hs_path(hs.HS_OP_BLOCK_SCORE_ATTN, hs.HS_F32, H, 576, 512, 64) == hs.HS_PATH_SIMT
+    args = [p, 64 * 576, 576, p, 576, p, 512, p, 1, T, 100, H, 576, 512, hs.HS_BF16, 0.0]
+    # block size, missing outputs, nb_stride below NBmax, missing v
+    assert L.hs_block_score_attn_fwd(*args, 8, p, p, p, 2, None, p, ws, None) == hs.HS_ERR_UNSUPPORTED
+    assert L.hs_block_score_attn_fwd(*args, 64, None, p, p, 2, None, p, ws, None) == hs.HS_ERR_INVALID_ARG
+    assert L.hs_block_score_attn_fwd(*args, 64, p, p, None, 2, None, p, ws, None) == hs.HS_ERR_INVALID_ARG
+    assert L.hs_block_score_attn_fwd(*args, 64, p, p, p, 1, None, p, ws, None) == hs.HS_ERR_INVALID_ARG
+    no_v = list(args)
+    no_v[5] = None
+    assert L.hs_block_score_attn_fwd(*no_v, 64, p, p, p, 2, None, p, ws, None) == hs.HS_ERR_INVALID_ARG
+    # no tokens: nothing to do
+    empty = list(args)
+    empty[9] = 0
+    assert L.hs_block_score_attn_fwd(*empty, 64, p, p, p, 2, None, None, 0, None) == hs.HS_OK
