@@ -3,8 +3,9 @@
 This package is the plain, slow, float64 definition of the four forward steps
 (block scoring, top-k block selection, block-sparse MQA attention and
 sliding-window MQA attention), of the full layer's forward that emits the
-block scores with its attention output, and of the backward of the two
-attention steps, which the CUDA library is checked against.
+block scores with its attention output, of the SWA layer that combines the
+window branch with the sparse branch on the shared KV, and of the backward
+of the two attention steps, which the CUDA library is checked against.
 
 It is test infrastructure: only the test-suite, the smoke check in
 ``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import it.
@@ -13,8 +14,9 @@ The CUDA product path never imports it and shares no code with it.
 Modules
 -------
 hysparse
-    Vectorised NumPy float64 implementation of the four steps and of the
-    full layer's fused forward (``full_layer_fwd``).
+    Vectorised NumPy float64 implementation of the four steps, of the full
+    layer's fused forward (``full_layer_fwd``) and of the SWA layer's two
+    branches combined (``swa_layer_fwd``).
 backward
     The gradient of the two attention steps (dq, dk, dv, sink gradient).
 loops
@@ -36,4 +38,5 @@ from .hysparse import (  # noqa: F401
     swa_mqa_fwd,
     dense_causal_fwd,
     full_layer_fwd,
+    swa_layer_fwd,
 )

@@ -67,6 +67,7 @@ __all__ = [
     "swa_mqa_fwd",
     "dense_causal_fwd",
     "full_layer_fwd",
+    "swa_layer_fwd",
 ]
 
 
@@ -410,3 +411,40 @@ def full_layer_fwd(q, k, v, cu_seqlens, block_size: int, scale=None, rows=None):
             acc = acc + np.exp(blse[i, h, :nb] - lse[i, h])
         score[i, :nb] = acc
     return {"out": out, "lse": lse, "block_lse": blse, "block_score": score}
+
+
+# ---------------------------------------------------------------------------
+# the HySparse SWA layer: window branch + sparse branch on the shared KV
+# ---------------------------------------------------------------------------
+
+def swa_layer_fwd(q, k, v, k_shared, v_shared, idx, cu_seqlens, window: int,
+                  block_size: int, sink_swa=None, sink_sparse=None, gate_swa=None,
+                  gate_sparse=None, scale=None, rows=None):
+    """Forward of the HySparse SWA layer ([HS] "What": NSA-style cooperating
+    structures; Copilot overview: the SWA kernel is the SWA layer's main
+    branch, the full layer produces the shared KV and the block indices;
+    [REV] MQA test review: the SWA layer consumes shared_kv in a sparse
+    branch).
+
+    Reading taken (the pages name the two branches, not how they combine):
+    as in NSA, each branch is its own softmax attention and the layer output
+    is their gated sum::
+
+        out[t,h] = gate_swa[t,h] * swa(q, k, v)[t,h]
+                 + gate_sparse[t,h] * sparse(q, k_shared, v_shared, idx)[t,h]
+
+    with the SWA layer's own queries q in both branches, each branch with its
+    own optional per-head sink, and a missing gate meaning 1 (a plain sum).
+    ``idx`` holds the block lists the full layer selected, one row per query
+    in ``rows`` order (as ``sparse_mqa_fwd``); gates are [T, H].  Returns
+    dict(out [R,H,Dv], lse_swa [R,H], lse_sparse [R,H]).
+    """
+    w = swa_mqa_fwd(q, k, v, cu_seqlens, window, sink=sink_swa, scale=scale, rows=rows)
+    sp = sparse_mqa_fwd(q, k_shared, v_shared, idx, cu_seqlens, block_size, sink=sink_sparse,
+                        scale=scale, rows=rows)
+    T = np.asarray(k).shape[0]
+    rr = _rows(rows, T)
+    gw = np.ones((rr.shape[0], w["out"].shape[1])) if gate_swa is None else _f64(gate_swa)[rr]
+    gs = np.ones_like(gw) if gate_sparse is None else _f64(gate_sparse)[rr]
+    out = gw[:, :, None] * w["out"] + gs[:, :, None] * sp["out"]
+    return {"out": out, "lse_swa": w["lse"], "lse_sparse": sp["lse"]}
