@@ -56,6 +56,8 @@ def parse():
                     help="skip the (separately timed) backward of the two attention steps")
     ap.add_argument("--no-full-layer", action="store_true",
                     help="skip the (separately timed) full layer's fused forward")
+    ap.add_argument("--no-swa-layer", action="store_true",
+                    help="skip the (separately timed) combined SWA layer")
     ap.add_argument("--cpu-rows", type=int, default=3072,
                     help="query rows of the oracle sample (cpu_baseline / reference arm)")
     return ap.parse_args()
@@ -462,6 +464,10 @@ def run_ours(args, wl, world, rank):
     full = None
     if not args.no_full_layer:
         full = run_full_layer(inp, wl, pk, flush, avg["score"])
+    layer = None
+    if not args.no_swa_layer:
+        layer = run_swa_layer(inp, wl, step, pk, flush, flops["sparse"] + flops["swa"],
+                              avg["sparse"] + avg["swa"])
 
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -482,8 +488,53 @@ def run_ours(args, wl, world, rank):
         "e2e": e2e,
         "backward": bwd,
         "full_layer": full,
+        "swa_layer": layer,
     }
     return res
+
+
+def run_swa_layer(inp, wl, step, pk, flush, flops, separate_ms, reps=3):
+    """The combined SWA layer (window branch + sparse branch, gated sum), not
+    part of the headline step: the step's q, k, v serve as both the layer's
+    own and the shared KV and the step's block lists as the full layer's;
+    per-(token, head) gates are uniform random.  CUDA-event time per call
+    with L2 flushed before each; algorithmic work = the two branches'."""
+    T, H = wl.total_tokens, wl.num_heads
+    dev = inp.q.device
+    g = torch.Generator(device=dev)
+    g.manual_seed(321)
+    gw = torch.rand((T, H), generator=g, device=dev)
+    gs = torch.rand((T, H), generator=g, device=dev)
+    out = torch.empty((T, H, wl.dv), device=dev, dtype=inp.q.dtype)
+    lw = torch.empty((T, H), device=dev, dtype=torch.float32)
+    ls = torch.empty_like(lw)
+
+    def fn():
+        hs.hs_swa_layer_fwd(inp.q, inp.k, inp.v, inp.k, inp.v, step.idx, inp.cu_seqlens,
+                            inp.max_seqlen, wl.window, wl.block_size, inp.sink, inp.sink, gw, gs,
+                            out=out, lse_swa=lw, lse_sparse=ls)
+
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for r in range(reps):
+        flush.fill_(r & 0xff)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    hs.poll_status(dev)
+    ms = statistics.mean(ts)
+    tf = flops / (ms / 1e3) / 1e12
+    return {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / pk["bf16_tflops"],
+            "algorithmic_flops": flops, "calls_timed": reps,
+            "separate_sparse_plus_swa_ms": separate_ms, "tokens_per_s": T / (ms / 1e3),
+            "path": "tcgen05" if hs.path(hs.HS_OP_SWA_LAYER, wl.dtype, H, wl.dk, wl.dv,
+                                         wl.block_size) == hs.HS_PATH_TCGEN05 else "simt",
+            "launches_per_call": 2}
 
 
 def run_full_layer(inp, wl, pk, flush, score_ms, reps=3):

@@ -171,6 +171,7 @@ int hs_path(int op, hs_dtype dtype, int num_heads, int dk, int dv, int block_siz
     case HS_OP_SPARSE_MQA:
     case HS_OP_SWA_MQA:
     case HS_OP_BLOCK_SCORE_ATTN:  // fused, or the attention then the score kernel
+    case HS_OP_SWA_LAYER:         // the sparse branch, then the window branch combining
       if (dtype == HS_BF16 && !g_force_simt.load() &&
           hs::tc_attention_supported(num_heads, dk, dv, block_size, op == HS_OP_SPARSE_MQA))
         return HS_PATH_TCGEN05;
@@ -425,6 +426,59 @@ hs_status hs_block_score_attn_fwd(const void* q, int64_t q_row_stride, int64_t q
                         total_tokens, max_seqlen, num_heads, dk, dtype, softmax_scale,
                         block_size, lse, block_score, nb_stride, block_lse, workspace,
                         workspace_bytes, stream);
+}
+
+hs_status hs_swa_layer_fwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                           const void* k, int64_t k_row_stride, const void* v,
+                           int64_t v_row_stride, const void* k_shared,
+                           int64_t k_shared_row_stride, const void* v_shared,
+                           int64_t v_shared_row_stride, const int32_t* cu_seqlens, int num_docs,
+                           int total_tokens, int max_seqlen, int num_heads, int dk, int dv,
+                           hs_dtype dtype, float softmax_scale, int window, const float* sink_swa,
+                           const int32_t* idx, int topk, int block_size,
+                           const float* sink_sparse, const float* gate_swa,
+                           const float* gate_sparse, void* out, float* lse_swa,
+                           float* lse_sparse, hs_stream_t stream) {
+  if (window < 1) return fail(HS_ERR_INVALID_ARG, "window %d < 1", window);
+  if (!valid_block(block_size))
+    return fail(HS_ERR_UNSUPPORTED, "block_size %d not in {16, 32, 64, 128}", block_size);
+  if (topk < 1 || topk > 256) return fail(HS_ERR_UNSUPPORTED, "topk %d not in [1, 256]", topk);
+  if (!idx) return fail(HS_ERR_INVALID_ARG, "idx is NULL");
+  if (!k_shared || !v_shared) return fail(HS_ERR_INVALID_ARG, "k_shared or v_shared is NULL");
+  if (k_shared_row_stride < dk)
+    return fail(HS_ERR_INVALID_ARG, "k_shared_row_stride %lld < dk", (long long)k_shared_row_stride);
+  if (v_shared_row_stride < dv)
+    return fail(HS_ERR_INVALID_ARG, "v_shared_row_stride %lld < dv", (long long)v_shared_row_stride);
+  if (!lse_sparse || !lse_swa) return fail(HS_ERR_INVALID_ARG, "lse_swa or lse_sparse is NULL");
+  // the window branch's own arguments, checked before the first launch
+  if (!k || !v) return fail(HS_ERR_INVALID_ARG, "k or v is NULL");
+  if (k_row_stride < dk) return fail(HS_ERR_INVALID_ARG, "k_row_stride %lld < dk",
+                                     (long long)k_row_stride);
+  if (v_row_stride < dv) return fail(HS_ERR_INVALID_ARG, "v_row_stride %lld < dv",
+                                     (long long)v_row_stride);
+  // the sparse branch over the shared KV, written to out
+  hs::AttnArgs sp{};
+  sp.idx = idx;
+  sp.topk = topk;
+  sp.block_size = block_size;
+  sp.window = 0;
+  hs_status r = attention_common(sp, true, q, q_row_stride, q_head_stride, k_shared,
+                                 k_shared_row_stride, v_shared, v_shared_row_stride, cu_seqlens,
+                                 num_docs, total_tokens, max_seqlen, num_heads, dk, dv, dtype,
+                                 softmax_scale, sink_sparse, out, lse_sparse, stream);
+  if (r != HS_OK) return r;
+  // the window branch, whose epilogue adds the gated sparse result from out
+  hs::AttnArgs w{};
+  w.idx = nullptr;
+  w.topk = 0;
+  w.block_size = 64;
+  w.window = window;
+  w.prev = out;
+  w.gate_own = gate_swa;
+  w.gate_prev = gate_sparse;
+  return attention_common(w, false, q, q_row_stride, q_head_stride, k, k_row_stride, v,
+                          v_row_stride, cu_seqlens, num_docs, total_tokens, max_seqlen,
+                          num_heads, dk, dv, dtype, softmax_scale, sink_swa, out, lse_swa, stream);
 }
 
 static hs_status backward_common(hs::BwdArgs& a, bool sparse, const void* q, int64_t qrs,

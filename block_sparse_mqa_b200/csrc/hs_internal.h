@@ -42,6 +42,12 @@ struct AttnArgs {
   const float* sink;   // may be null
   void* out;
   float* lse;
+  // optional combining epilogue (the SWA layer): out = gate_own * result +
+  // gate_prev * prev; prev [T, H, Dv] of dtype, may alias out; gates [T, H]
+  // fp32 or null (= 1).  prev == null: plain output.
+  const void* prev = nullptr;
+  const float* gate_own = nullptr;
+  const float* gate_prev = nullptr;
 };
 
 // The full layer's fused forward (after host validation): dense causal

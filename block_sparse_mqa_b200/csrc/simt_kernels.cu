@@ -228,10 +228,18 @@ simt_attention_kernel(AttnArgs a) {
     inv = em / denom;
   }
   T* o = reinterpret_cast<T*>(a.out) + ((int64_t)t * p.num_heads + h) * Dv;
+  const int64_t th = (int64_t)t * p.num_heads + h;
+  const float gown = a.gate_own ? __ldg(a.gate_own + th) : 1.f;
+  const float gprev = a.gate_prev ? __ldg(a.gate_prev + th) : 1.f;
+  const T* pr = a.prev ? reinterpret_cast<const T*>(a.prev) + th * Dv : nullptr;
 #pragma unroll
   for (int r = 0; r < kMaxDvPerThread; ++r) {
     const int d = tid + r * kAttnThreads;
-    if (d < Dv) o[d] = from_f32<T>(acc[r] * inv);
+    if (d < Dv) {
+      float x = acc[r] * inv * gown;
+      if (pr) x = fmaf(gprev, to_f32<T>(pr[d]), x);  // read before the write below
+      o[d] = from_f32<T>(x);
+    }
   }
   if (tid == 0) a.lse[(int64_t)t * p.num_heads + h] = lse;
 }

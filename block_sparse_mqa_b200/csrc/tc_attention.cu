@@ -79,7 +79,8 @@ constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kRescaleLog2 = 8.f;  // raise the running max only past 2^8
 
-constexpr int kModeSwa = 0, kModeSparse = 1, kModeFull = 2;
+// kModeSwaLayer: the window attention with the combining epilogue
+constexpr int kModeSwa = 0, kModeSparse = 1, kModeFull = 2, kModeSwaLayer = 3;
 
 struct AttnParams {
   const int32_t* cu;
@@ -99,6 +100,11 @@ struct AttnParams {
   int nbmax, nb_stride;
   float* block_score;  // [T, nb_stride]
   float* block_lse;    // [T, kH, nb_stride] or null
+  // combining epilogue (the SWA layer): out = gate_own * this attention +
+  // gate_prev * prev, prev [T, kH, Dv] bf16 (may be out itself); null = off
+  const __nv_bfloat16* prev;
+  const float* gate_own;   // [T, kH] or null (= 1)
+  const float* gate_prev;  // [T, kH] or null (= 1)
 };
 
 struct Shared {
@@ -112,6 +118,7 @@ struct Shared {
   float red[2][4][32];       // [warpgroup][warp][lane] partial reductions
   float bsum[2][4][32];      // [warpgroup][warp][head] one tile's exp sums (full layer)
   float lse2[kH];            // row LSE per head, log2 units (full layer)
+  float gprev[kH];           // gate of prev per head (combining epilogue)
   float mrun[kH];            // running max per head (log2 domain)
   float alpha[kH];           // rescale factor per head
   float lsum[kH];            // output multiplier per head
@@ -254,6 +261,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap qmap, const AttnParams p) {
   constexpr bool kSparse = kMode == kModeSparse;
   constexpr bool kFull = kMode == kModeFull;
+  constexpr bool kCombine = kMode == kModeSwaLayer;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -554,6 +562,11 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         }
         if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
       }
+      if (kCombine) {  // this warpgroup's rows of prev towards L2 for the epilogue
+        const char* pb = reinterpret_cast<const char*>(p.prev + ((int64_t)t * kH + hb) * dvs);
+        for (int off = r * 128; off < 32 * dvs * 2; off += 128 * 128)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(pb + off));
+      }
       float lpart[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) lpart[k] = 0.f;
@@ -631,11 +644,16 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           sh->bsum[wg][g4][lane] = tr_sum(x);
           m_used = sh->mrun[hb + lane];
         }
-        // P^T may be rewritten once PV of the previous tile has read it
+        // P^T may be rewritten once PV of the previous tile has read it, and
+        // on a token's first tile once BOTH warpgroups have finished staging
+        // the previous token's output in the same buffer (each warpgroup's
+        // staging half spans rows that hold the other warpgroup's P^T columns)
         if (i > 0) {
           if (!mbar_wait(&sh->pvdone, npv & 1, lim)) { ok = false; break; }
           ++npv;
           tc_fence_after();
+        } else if (ntok > 0) {
+          if (!mbar_wait(&sh->oempty, (ntok - 1) & 1, lim)) { ok = false; break; }
         }
         if (resc) {  // rare: some head's running max rose; rescale its O^T columns
 #pragma unroll 1
@@ -678,6 +696,10 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         const float M = fmaxf(m, sk);
         const float den = l * fast_exp2(m - M) + fast_exp2(sk - M);
         sh->lsum[hh] = fast_exp2(m - M) / den;
+        if (kCombine) {
+          if (p.gate_own) sh->lsum[hh] *= __ldg(p.gate_own + (int64_t)t * kH + hh);
+          sh->gprev[hh] = p.gate_prev ? __ldg(p.gate_prev + (int64_t)t * kH + hh) : 1.f;
+        }
         sh->lse2[hh] = M + fast_log2(den);
         p.lse[(int64_t)t * kH + hh] = sh->lse2[hh] * kLn2;
       }
@@ -699,6 +721,20 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
         for (int k = 0; k < 32; ++k) ls[k] = sh->lsum[hb + k];
         for (int c = 0; c < p.nvc; ++c) {
+          // combining epilogue: the 16-byte units of prev this thread will
+          // overwrite, loaded before the TMEM read so the latency overlaps
+          uint4 pv[4];
+          if (kCombine) {
+            const __nv_bfloat16* pbase = p.prev + ((int64_t)t * kH + hb) * dvs;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const int u = r + 128 * q4;
+              const int col = c * 128 + (u & 15) * 8;
+              pv[q4] = col < dvs ? *reinterpret_cast<const uint4*>(
+                                       pbase + (int64_t)(u >> 4) * dvs + col)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
           uint32_t w[32];
           tmem_ld32(lane_base + c * kH + hb, w);
           tmem_ld_wait();
@@ -707,13 +743,36 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           for (int k = 0; k < 32; ++k)
             stage[k * 128 + r] = __float2bfloat16_rn(__uint_as_float(w[k]) * ls[k]);
           named_bar(1 + wg, 128);
+          if (kCombine) {
+            // the gated other branch joins in fp32
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int u = r + 128 * q4;  // 16-byte unit: head u / 16, dv 8 (u % 16)
-            const uint4 v = reinterpret_cast<const uint4*>(stage)[u];
-            const int col = c * 128 + (u & 15) * 8;
-            if (col < dvs)  // a last chunk half past Dv holds zero rows
-              *reinterpret_cast<uint4*>(obase + (int64_t)(u >> 4) * dvs + col) = v;
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const int u = r + 128 * q4;
+              const int col = c * 128 + (u & 15) * 8;
+              if (col < dvs) {
+                uint4 v = reinterpret_cast<const uint4*>(stage)[u];
+                const float g = sh->gprev[hb + (u >> 4)];
+                uint32_t* vw = reinterpret_cast<uint32_t*>(&v);
+                const uint32_t* pw = reinterpret_cast<const uint32_t*>(&pv[q4]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vw[e]));
+                  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[e]));
+                  __nv_bfloat162 o = __floats2bfloat162_rn(fmaf(g, b.x, a.x), fmaf(g, b.y, a.y));
+                  vw[e] = *reinterpret_cast<uint32_t*>(&o);
+                }
+                *reinterpret_cast<uint4*>(obase + (int64_t)(u >> 4) * dvs + col) = v;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const int u = r + 128 * q4;  // 16-byte unit: head u / 16, dv 8 (u % 16)
+              const uint4 v = reinterpret_cast<const uint4*>(stage)[u];
+              const int col = c * 128 + (u & 15) * 8;
+              if (col < dvs)  // a last chunk half past Dv holds zero rows
+                *reinterpret_cast<uint4*>(obase + (int64_t)(u >> 4) * dvs + col) = v;
+            }
           }
           named_bar(1 + wg, 128);
         }
@@ -771,7 +830,8 @@ bool tc_attention_supported(int num_heads, int dk, int dv, int block_size, bool 
 bool tc_attention_eligible(const AttnArgs& a) {
   const Problem& p = a.p;
   auto al16 = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; };
-  return al16(p.q) && al16(p.k) && al16(p.v) && al16(a.out) && p.q_row_stride % 8 == 0 &&
+  return al16(p.q) && al16(p.k) && al16(p.v) && al16(a.out) && al16(a.prev) &&
+         p.q_row_stride % 8 == 0 &&
          p.q_head_stride % 8 == 0 && p.k_row_stride % 8 == 0 && p.v_row_stride % 8 == 0;
 }
 
@@ -824,10 +884,14 @@ cudaError_t launch_mode(const AttnArgs& a, int mode, const FullArgs* fa, long lo
   ap.nb_stride = fa ? fa->nb_stride : 0;
   ap.block_score = fa ? fa->block_score : nullptr;
   ap.block_lse = fa ? fa->block_lse : nullptr;
+  ap.prev = static_cast<const __nv_bfloat16*>(a.prev);
+  ap.gate_own = a.gate_own;
+  ap.gate_prev = a.gate_prev;
   const int grid = p.total_tokens < sm_count() ? p.total_tokens : sm_count();
-  auto kern = mode == kModeSparse ? tc_attention_kernel<kModeSparse>
-              : mode == kModeFull ? tc_attention_kernel<kModeFull>
-                                  : tc_attention_kernel<kModeSwa>;
+  auto kern = mode == kModeSparse   ? tc_attention_kernel<kModeSparse>
+              : mode == kModeFull   ? tc_attention_kernel<kModeFull>
+              : mode == kModeSwaLayer ? tc_attention_kernel<kModeSwaLayer>
+                                    : tc_attention_kernel<kModeSwa>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -839,7 +903,9 @@ cudaError_t launch_mode(const AttnArgs& a, int mode, const FullArgs* fa, long lo
 
 cudaError_t launch_tc_attention(const AttnArgs& a, bool sparse, long long wait_limit,
                                 cudaStream_t s) {
-  return launch_mode(a, sparse ? kModeSparse : kModeSwa, nullptr, wait_limit, s);
+  if (a.prev && sparse) return cudaErrorInvalidValue;  // combining is a window-branch mode
+  return launch_mode(a, sparse ? kModeSparse : a.prev ? kModeSwaLayer : kModeSwa, nullptr,
+                     wait_limit, s);
 }
 
 bool tc_full_supported(int num_heads, int dk, int dv, int block_size) {

@@ -38,6 +38,7 @@ HS_OP_SWA_MQA = 3
 HS_OP_SPARSE_MQA_BWD = 4
 HS_OP_SWA_MQA_BWD = 5
 HS_OP_BLOCK_SCORE_ATTN = 6
+HS_OP_SWA_LAYER = 7
 
 HS_PATH_SIMT = 0
 HS_PATH_TCGEN05 = 1
@@ -49,7 +50,7 @@ EXPORTS = (
     "hs_workspace_size", "hs_path", "hs_poll_status", "hs_set_force_simt",
     "hs_selftest_wait", "hs_status_string", "hs_last_error", "hs_version",
     "hs_block_score_static", "hs_sparse_mqa_bwd", "hs_swa_mqa_bwd",
-    "hs_block_score_attn_fwd",
+    "hs_block_score_attn_fwd", "hs_swa_layer_fwd",
 )
 
 
@@ -95,6 +96,9 @@ def lib() -> ctypes.CDLL:
     L.hs_block_score_attn_fwd.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _int, _int,
                                           _int, _int, _int, _int, _int, _flt, _int, _vp, _vp,
                                           _vp, _int, _vp, _vp, _szt, _vp]
+    L.hs_swa_layer_fwd.argtypes = [_vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _i64, _vp, _i64,
+                                   _vp, _int, _int, _int, _int, _int, _int, _int, _flt, _int,
+                                   _vp, _vp, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.hs_workspace_size.argtypes = [_int] * 9
     L.hs_workspace_size.restype = _szt
     L.hs_path.argtypes = [_int] * 6
@@ -109,7 +113,7 @@ def lib() -> ctypes.CDLL:
     L.hs_last_error.restype = ctypes.c_char_p
     for fn in ("hs_block_score", "hs_select_topk", "hs_sparse_mqa_fwd", "hs_swa_mqa_fwd",
                "hs_poll_status", "hs_block_score_static", "hs_sparse_mqa_bwd",
-               "hs_swa_mqa_bwd", "hs_block_score_attn_fwd"):
+               "hs_swa_mqa_bwd", "hs_block_score_attn_fwd", "hs_swa_layer_fwd"):
         getattr(L, fn).restype = _int
     _lib = L
     return L
@@ -344,6 +348,39 @@ def hs_block_score_attn_fwd(q, k, v, cu_seqlens, max_seqlen: int, block_size: in
         _ptr(o), _ptr(l), _ptr(bs), bs.stride(0), _ptr(blse), _ptr(workspace),
         0 if workspace is None else workspace.numel(), _stream(dev)))
     return o, l, bs, blse
+
+
+def hs_swa_layer_fwd(q, k, v, k_shared, v_shared, idx, cu_seqlens, max_seqlen: int, window: int,
+                     block_size: int, sink_swa=None, sink_sparse=None, gate_swa=None,
+                     gate_sparse=None, softmax_scale: float = 0.0, out=None, lse_swa=None,
+                     lse_sparse=None):
+    """The SWA layer: window attention over its own k, v plus the sparse
+    branch over the full layer's k_shared, v_shared and block lists idx,
+    combined as gate_swa * window + gate_sparse * sparse (missing gates = 1).
+    Returns (out [T,H,Dv] in q's dtype, lse_swa [T,H], lse_sparse [T,H])."""
+    _need_cuda(q, k, v, k_shared, v_shared, idx, cu_seqlens, sink_swa, sink_sparse, gate_swa,
+               gate_sparse)
+    qrs, qhs, krs = _qk_strides(q, k)
+    _, _, ksrs = _qk_strides(q, k_shared)
+    for name, t in (("v", v), ("v_shared", v_shared)):
+        if t.dim() != 2 or t.stride(1) != 1:
+            raise ValueError(name + " must be [T, Dv] with contiguous rows")
+    if idx.dtype != torch.int32 or not idx.is_contiguous():
+        raise ValueError("idx must be contiguous int32 [T, topk]")
+    T, H, Dk = q.shape
+    for name, g in (("gate_swa", gate_swa), ("gate_sparse", gate_sparse)):
+        if g is not None and (g.dtype != torch.float32 or tuple(g.shape) != (T, H) or
+                              not g.is_contiguous()):
+            raise ValueError(name + " must be contiguous float32 [T, H]")
+    o, lw = _attn_out(q, v, out, lse_swa)
+    ls = lse_sparse if lse_sparse is not None else torch.empty_like(lw)
+    _check(lib().hs_swa_layer_fwd(
+        _ptr(q), qrs, qhs, _ptr(k), krs, _ptr(v), v.stride(0), _ptr(k_shared), ksrs,
+        _ptr(v_shared), v_shared.stride(0), _ptr(cu_seqlens), cu_seqlens.numel() - 1, T,
+        int(max_seqlen), H, Dk, v.shape[1], _dtype_code(q), float(softmax_scale), int(window),
+        _ptr(sink_swa), _ptr(idx), idx.shape[1], int(block_size), _ptr(sink_sparse),
+        _ptr(gate_swa), _ptr(gate_sparse), _ptr(o), _ptr(lw), _ptr(ls), _stream(q.device)))
+    return o, lw, ls
 
 
 def _bwd_prep(q, k, v, out, lse, dout, cu_seqlens, sink, op, max_seqlen, grads, workspace):

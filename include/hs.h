@@ -20,7 +20,9 @@
  *
  * hs_block_score_attn_fwd is the full layer's forward: dense causal
  * attention that emits step 1's outputs from the same pass, replacing
- * hs_block_score where the model runs that layer anyway.
+ * hs_block_score where the model runs that layer anyway.  hs_swa_layer_fwd
+ * is the SWA layer: its window attention plus a block-sparse branch over the
+ * full layer's shared KV, combined.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -99,7 +101,8 @@ typedef enum hs_op {
   HS_OP_SWA_MQA = 3,
   HS_OP_SPARSE_MQA_BWD = 4,
   HS_OP_SWA_MQA_BWD = 5,
-  HS_OP_BLOCK_SCORE_ATTN = 6
+  HS_OP_BLOCK_SCORE_ATTN = 6,
+  HS_OP_SWA_LAYER = 7
 } hs_op;
 
 /* Kernel family a call will use, as returned by hs_path(). */
@@ -326,6 +329,46 @@ hs_status hs_block_score_attn_fwd(const void* q, int64_t q_row_stride, int64_t q
                                   void* out, float* lse, float* block_score, int nb_stride,
                                   float* block_lse, void* workspace, size_t workspace_bytes,
                                   hs_stream_t stream);
+
+/*
+ * The HySparse SWA layer: window branch + sparse branch on the shared KV.
+ * Source: pull request 1470, "What" (NSA-style, three cooperating
+ * structures) and Copilot overview (the SWA kernel is wired into the SWA
+ * layer's main branch; the full layer produces the shared KV and the block
+ * indices); review of pull request 1453 (the SWA layer consumes shared_kv
+ * in a sparse branch).  The pages do not say how the branches combine; as in
+ * NSA, each branch is its own softmax and the output is their gated sum:
+ *   out[t,h] = gate_swa[t,h]    * swa(q, k, v; window, sink_swa)[t,h]
+ *            + gate_sparse[t,h] * sparse(q, k_shared, v_shared; idx, sink_sparse)[t,h]
+ * with the two branches defined exactly as hs_swa_mqa_fwd and
+ * hs_sparse_mqa_fwd, over the same queries q (the SWA layer's own).
+ *
+ *   k, v                [T, Dk], [T, Dv]: the SWA layer's own keys / values.
+ *   k_shared, v_shared  [T, Dk], [T, Dv]: the full layer's keys / values
+ *                       (same dims; v_shared may alias k_shared).
+ *   idx                 [T, topk]: the full layer's block lists (the rule
+ *                       of hs_sparse_mqa_fwd).
+ *   gate_swa, gate_sparse  [T, H] fp32, or NULL for 1 (then a plain sum).
+ *   out                 [T, H, Dv] of `dtype`, contiguous, output.
+ *   lse_swa, lse_sparse [T, H] fp32 outputs: each branch's lse (with its sink).
+ * No workspace.  The call runs the sparse branch into `out`, then the window
+ * attention whose epilogue adds the gated sparse result it reads back from
+ * `out` (fp32 arithmetic, one rounding to bf16 for the sum's window part and
+ * one for the sum); 16-byte-aligned bf16 inputs with 64 heads use the
+ * tcgen05 kernels for both.
+ */
+hs_status hs_swa_layer_fwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
+                           const void* k, int64_t k_row_stride,
+                           const void* v, int64_t v_row_stride,
+                           const void* k_shared, int64_t k_shared_row_stride,
+                           const void* v_shared, int64_t v_shared_row_stride,
+                           const int32_t* cu_seqlens, int num_docs, int total_tokens,
+                           int max_seqlen, int num_heads, int dk, int dv, hs_dtype dtype,
+                           float softmax_scale, int window, const float* sink_swa,
+                           const int32_t* idx, int topk, int block_size,
+                           const float* sink_sparse, const float* gate_swa,
+                           const float* gate_sparse, void* out, float* lse_swa,
+                           float* lse_sparse, hs_stream_t stream);
 
 /*
  * Step 1 for callers that cannot allocate device memory.

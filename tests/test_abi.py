@@ -185,3 +185,27 @@ def test_full_layer_rejects_bad_arguments():
     empty = list(args)
     empty[9] = 0
     assert L.hs_block_score_attn_fwd(*empty, 64, p, p, p, 2, None, None, 0, None) == hs.HS_OK
+
+
+def test_swa_layer_rejects_bad_arguments():
+    L = hs.lib()
+    p = ctypes.c_void_p(256)
+    T, H = 100, 64
+    assert L.hs_path(hs.HS_OP_SWA_LAYER, hs.HS_BF16, H, 576, 512, 64) == hs.HS_PATH_TCGEN05
+    assert L.hs_workspace_size(hs.HS_OP_SWA_LAYER, T, 1, 100, H, 576, 512, hs.HS_BF16, 64) == 0
+    head = [p, 64 * 576, 576, p, 576, p, 512]          # q, k, v
+    shared = [p, 576, p, 512]                          # k_shared, v_shared
+    common = [p, 1, T, 100, H, 576, 512, hs.HS_BF16, 0.0]
+    def call(head=head, shared=shared, window=64, idx=p, topk=4, B=64, outs=(p, p, p)):
+        return L.hs_swa_layer_fwd(*head, *shared, *common, window, None, idx, topk, B, None,
+                                  None, None, *outs, None)
+    assert call(window=0) == hs.HS_ERR_INVALID_ARG
+    assert call(B=24) == hs.HS_ERR_UNSUPPORTED
+    assert call(topk=0) == hs.HS_ERR_UNSUPPORTED
+    assert call(idx=None) == hs.HS_ERR_INVALID_ARG
+    assert call(shared=[None, 576, p, 512]) == hs.HS_ERR_INVALID_ARG
+    assert call(shared=[p, 100, p, 512]) == hs.HS_ERR_INVALID_ARG
+    assert call(head=[p, 64 * 576, 576, p, 576, None, 512]) == hs.HS_ERR_INVALID_ARG
+    assert call(head=[p, 64 * 576, 576, p, 576, p, 500]) == hs.HS_ERR_INVALID_ARG
+    assert call(outs=(p, None, p)) == hs.HS_ERR_INVALID_ARG
+    assert call(outs=(p, p, None)) == hs.HS_ERR_INVALID_ARG
