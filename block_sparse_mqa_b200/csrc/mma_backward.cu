@@ -18,9 +18,10 @@
 // partial sums are added in rank order through distributed shared memory
 // (a tile every query selects, such as a document's first block, is then
 // spread over four SMs).  Per member token t (all 64 heads):
-//   S^T [32 keys x 64 heads]  = K_tile . q_t^T      (each warp one 16x8 tile)
-//   dP^T[32 x 64]             = V_tile . dout_t^T
-//   P^T, dS^T (bf16)          -> shared memory
+//   S^T [32 keys x 64 heads]  = K_tile . q_t^T      (warps 0-7, 16x16 each)
+//   dP^T[32 x 64]             = V_tile . dout_t^T   (warps 8-15, 16x16 each)
+//   P^T, dS^T (bf16)          -> shared memory      (dP^T passed to the S^T
+//                                                    warps through it, fp32)
 //   dK[32 x Dk] += dS^T . q_t,  dV[32 x Dv] += P^T . dout_t   (registers)
 // Sums run in a fixed order: results are deterministic.
 
@@ -72,6 +73,15 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 __device__ __forceinline__ void ldsm_x2_trans(uint32_t& b0, uint32_t& b1, uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
                : "=r"(b0), "=r"(b1)
+               : "r"(addr));
+}
+
+// Four 8x8 bf16 matrices, row addresses from lanes 8i..8i+7 for matrix i
+// (not transposed): the A fragment of an m16n8k16 MMA (rows 0-15 x k 0-15),
+// or the B fragments of two n8 tiles stored as [n][k] rows.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(addr));
 }
 
@@ -175,6 +185,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_mma_kernel(const MmaBwdP
   const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(P.q);
   const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(P.k);
   const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(P.v);
+  // Score phase: warp w < 8 computes S^T, warp w + 8 the dP^T block at the
+  // same place: keys 16 mt.., heads 16 np.. (two n8 tiles sharing each A
+  // fragment; ldmatrix for A and B).  dP^T goes to the S^T warp through an
+  // fp32 tile [kKT][kDP] laid over the P^T / dS^T buffers.
+  const bool s_warp = warp < 8;
+  const int mt = (warp >> 2) & 1, np = warp & 3;
+  constexpr int kDP = 72;  // fp32 row stride of the dP^T hand-over tile
+  static_assert(kKT * kDP * 4 <= 2 * kKT * kPS * 2, "dP tile must fit the P / dS buffers");
+  float* dpx = reinterpret_cast<float*>(Ps);
+  const uint32_t a_sc = (uint32_t)__cvta_generic_to_shared(s_warp ? Kt : Vt) +
+                        (uint32_t)(((mt * 16 + (lane & 15)) * (s_warp ? KS : VS) +
+                                    (lane >> 4) * 8) * 2);
+  const uint32_t b_sc = (s_warp ? qs_base : ds_base) +
+                        (uint32_t)(((np * 16 + (lane & 7) + ((lane >> 4) << 3)) *
+                                        (s_warp ? KS : VS) +
+                                    ((lane >> 3) & 1) * 8) * 2);
+  const int kend_sc = s_warp ? dk : dv;
   // The CTAs of a cluster share one key tile: each scans every candidate
   // (so all see the same member list) and takes every csize-th member; their
   // partial sums are added in rank order through distributed shared memory.
@@ -245,39 +272,59 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_mma_kernel(const MmaBwdP
           }
           cp_async_wait_all();
           __syncthreads();
-          // S^T and dP^T for keys wm*16.. x heads wn*8..
-          float sc[4] = {0.f, 0.f, 0.f, 0.f}, dp[4] = {0.f, 0.f, 0.f, 0.f};
-          {
-            const __nv_bfloat16* ka = Kt + (wm * 16 + g) * KS + 2 * tig;
-            const __nv_bfloat16* qb = Qs + (wn * 8 + g) * KS + 2 * tig;
-            for (int k0 = 0; k0 < dk; k0 += 16) {
-              const uint32_t af[4] = {lds32(ka + k0), lds32(ka + 8 * KS + k0), lds32(ka + k0 + 8),
-                                      lds32(ka + 8 * KS + k0 + 8)};
-              mma16816(sc, af, lds32(qb + k0), lds32(qb + k0 + 8));
-            }
-            const __nv_bfloat16* va = Vt + (wm * 16 + g) * VS + 2 * tig;
-            const __nv_bfloat16* db = Ds + (wn * 8 + g) * VS + 2 * tig;
-            for (int k0 = 0; k0 < dv; k0 += 16) {
-              const uint32_t af[4] = {lds32(va + k0), lds32(va + 8 * VS + k0), lds32(va + k0 + 8),
-                                      lds32(va + 8 * VS + k0 + 8)};
-              mma16816(dp, af, lds32(db + k0), lds32(db + k0 + 8));
+          // S^T (warps 0-7) or dP^T (warps 8-15) for keys 16 mt.. x heads 16 np..
+          float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          for (int k0 = 0; k0 < kend_sc; k0 += 16) {
+            uint32_t af[4], bf[4];
+            ldsm_x4(af, a_sc + (uint32_t)(k0 * 2));
+            ldsm_x4(bf, b_sc + (uint32_t)(k0 * 2));
+            mma16816(acc2[0], af, bf[0], bf[1]);
+            mma16816(acc2[1], af, bf[2], bf[3]);
+          }
+          const int r0 = mt * 16 + g;
+          if (!s_warp) {  // hand dP^T over (the P^T / dS^T buffers are free here)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int h = np * 16 + 8 * j + 2 * tig;
+              *reinterpret_cast<float2*>(dpx + r0 * kDP + h) = make_float2(acc2[j][0], acc2[j][1]);
+              *reinterpret_cast<float2*>(dpx + (r0 + 8) * kDP + h) =
+                  make_float2(acc2[j][2], acc2[j][3]);
             }
           }
-          // P^T = exp(s - lse) on member keys, dS^T = P^T (dP^T - delta)
-          {
-            const int r0 = wm * 16 + g, h0 = wn * 8 + 2 * tig;
-            float pv[4], dsv[4];
+          __syncthreads();
+          float dpv[2][4];
+          if (s_warp) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int key = r0 + ((q & 2) ? 8 : 0), head = h0 + (q & 1);
-              const float pr = ((mk >> key) & 1u) ? expf(sc[q] * scale - lse_s[head]) : 0.f;
-              pv[q] = pr;
-              dsv[q] = pr * (dp[q] - del_s[head]);
+            for (int j = 0; j < 2; ++j) {
+              const int h = np * 16 + 8 * j + 2 * tig;
+              const float2 lo = *reinterpret_cast<const float2*>(dpx + r0 * kDP + h);
+              const float2 hi = *reinterpret_cast<const float2*>(dpx + (r0 + 8) * kDP + h);
+              dpv[j][0] = lo.x;
+              dpv[j][1] = lo.y;
+              dpv[j][2] = hi.x;
+              dpv[j][3] = hi.y;
             }
-            *reinterpret_cast<uint32_t*>(Ps + r0 * kPS + h0) = pack_bf16(pv[0], pv[1]);
-            *reinterpret_cast<uint32_t*>(Ps + (r0 + 8) * kPS + h0) = pack_bf16(pv[2], pv[3]);
-            *reinterpret_cast<uint32_t*>(Ss + r0 * kPS + h0) = pack_bf16(dsv[0], dsv[1]);
-            *reinterpret_cast<uint32_t*>(Ss + (r0 + 8) * kPS + h0) = pack_bf16(dsv[2], dsv[3]);
+          }
+          __syncthreads();  // every dP^T value read before P^T / dS^T overwrite the tile
+          // P^T = exp(s - lse) on member keys, dS^T = P^T (dP^T - delta)
+          if (s_warp) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int h0 = np * 16 + 8 * j + 2 * tig;
+              float pv[4], dsv[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int key = r0 + ((q & 2) ? 8 : 0), head = h0 + (q & 1);
+                const float pr =
+                    ((mk >> key) & 1u) ? expf(acc2[j][q] * scale - lse_s[head]) : 0.f;
+                pv[q] = pr;
+                dsv[q] = pr * (dpv[j][q] - del_s[head]);
+              }
+              *reinterpret_cast<uint32_t*>(Ps + r0 * kPS + h0) = pack_bf16(pv[0], pv[1]);
+              *reinterpret_cast<uint32_t*>(Ps + (r0 + 8) * kPS + h0) = pack_bf16(pv[2], pv[3]);
+              *reinterpret_cast<uint32_t*>(Ss + r0 * kPS + h0) = pack_bf16(dsv[0], dsv[1]);
+              *reinterpret_cast<uint32_t*>(Ss + (r0 + 8) * kPS + h0) = pack_bf16(dsv[2], dsv[3]);
+            }
           }
           __syncthreads();
           // dK += dS^T . q_t and dV += P^T . dout_t over the 64 heads
@@ -358,19 +405,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_mma_kernel(const MmaBwdP
 // Query-major: one CTA per token t with q_t and dout_t (all heads) resident;
 // the token's key set in tiles of at most 32 keys that never cross a block
 // (SWA: the window).  Per tile:
-//   S [64 heads x 32 keys] = q_t . K_tile^T,  dP = dout_t . V_tile^T
-//       (16 warps: one 16 x 8 tile each)
+//   S [64 heads x 32 keys] = q_t . K_tile^T   (warps 0-7, 16 x 16 each)
+//   dP = dout_t . V_tile^T                    (warps 8-15, 16 x 16 each;
+//       handed to the S warps through an fp32 tile)
 //   dS = P (dP - delta) -> shared memory (bf16, [head][key])
 //   dQ [64 x Dk] += dS . K_tile   (registers: warp w owns heads 16 (w / 4)..
 //       and every fourth 8-column tile from w % 4)
 constexpr int kDS = kKT + kPad;  // row stride of the dS tile
 constexpr int kMaxNQ = 18;       // Dk / 32 n-tiles per warp (Dk <= 576)
 
+constexpr int kDQP = kKT + 8;    // fp32 row stride of the dP hand-over tile
+
 inline size_t mma_dq_smem_bytes(int dk, int dv) {
   const int KS = dk + kPad, VS = dv + kPad;
   return 2 * ((size_t)kH * KS + (size_t)kH * VS + (size_t)kKT * KS + (size_t)kKT * VS +
               (size_t)kH * kDS) +
-         4 * 2 * (size_t)kH + 4 * 256;
+         4 * (size_t)kH * kDQP + 4 * 2 * (size_t)kH + 4 * 256;
 }
 
 template <bool kSparse>
@@ -384,7 +434,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_mma_kernel(const MmaBwdPar
   __nv_bfloat16* Kt = Ds + kH * VS;                              // [kKT][KS]
   __nv_bfloat16* Vt = Kt + kKT * KS;                             // [kKT][VS]
   __nv_bfloat16* Sd = Vt + kKT * VS;                             // [kH][kDS] dS
-  float* lse_s = reinterpret_cast<float*>(Sd + kH * kDS);
+  float* dpx = reinterpret_cast<float*>(Sd + kH * kDS);          // [kH][kDQP] dP
+  float* lse_s = dpx + kH * kDQP;
   float* del_s = lse_s + kH;
   int* blist = reinterpret_cast<int*>(del_s + kH);               // [256]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tig = lane & 3;
@@ -396,6 +447,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_mma_kernel(const MmaBwdPar
   const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(P.q);
   const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(P.k);
   const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(P.v);
+  // Score phase: warp w < 8 computes S, warp w + 8 dP at the same place:
+  // heads 16 mh.., keys 16 nk.. (two n8 tiles sharing each A fragment).
+  const bool s_warp = warp < 8;
+  const int mh = (warp >> 1) & 3, nk = warp & 1;
+  const uint32_t a_sc = (uint32_t)__cvta_generic_to_shared(s_warp ? Qs : Ds) +
+                        (uint32_t)(((mh * 16 + (lane & 15)) * (s_warp ? KS : VS) +
+                                    (lane >> 4) * 8) * 2);
+  const uint32_t b_sc = (uint32_t)__cvta_generic_to_shared(s_warp ? Kt : Vt) +
+                        (uint32_t)(((nk * 16 + (lane & 7) + ((lane >> 4) << 3)) *
+                                        (s_warp ? KS : VS) +
+                                    ((lane >> 3) & 1) * 8) * 2);
+  const int kend_sc = s_warp ? dk : dv;
   for (int t = blockIdx.x; t < P.total_tokens; t += gridDim.x) {
     int bos, eos;
     if (!find_doc(P.cu_seqlens, P.num_docs, P.total_tokens, P.max_seqlen, t, bos, eos, P.status))
@@ -439,34 +502,42 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_mma_kernel(const MmaBwdPar
         copy_rows(Vt, VS, vg + (int64_t)j0 * P.v_row_stride, P.v_row_stride, n, dv, kKT);
         cp_async_wait_all();
         __syncthreads();
-        float sc[4] = {0.f, 0.f, 0.f, 0.f}, dp[4] = {0.f, 0.f, 0.f, 0.f};
-        {
-          const __nv_bfloat16* qa = Qs + (wm * 16 + g) * KS + 2 * tig;
-          const __nv_bfloat16* kb = Kt + (wn * 8 + g) * KS + 2 * tig;
-          for (int k0 = 0; k0 < dk; k0 += 16) {
-            const uint32_t af[4] = {lds32(qa + k0), lds32(qa + 8 * KS + k0), lds32(qa + k0 + 8),
-                                    lds32(qa + 8 * KS + k0 + 8)};
-            mma16816(sc, af, lds32(kb + k0), lds32(kb + k0 + 8));
-          }
-          const __nv_bfloat16* da = Ds + (wm * 16 + g) * VS + 2 * tig;
-          const __nv_bfloat16* vb = Vt + (wn * 8 + g) * VS + 2 * tig;
-          for (int k0 = 0; k0 < dv; k0 += 16) {
-            const uint32_t af[4] = {lds32(da + k0), lds32(da + 8 * VS + k0), lds32(da + k0 + 8),
-                                    lds32(da + 8 * VS + k0 + 8)};
-            mma16816(dp, af, lds32(vb + k0), lds32(vb + k0 + 8));
+        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        for (int k0 = 0; k0 < kend_sc; k0 += 16) {
+          uint32_t af[4], bf[4];
+          ldsm_x4(af, a_sc + (uint32_t)(k0 * 2));
+          ldsm_x4(bf, b_sc + (uint32_t)(k0 * 2));
+          mma16816(acc2[0], af, bf[0], bf[1]);
+          mma16816(acc2[1], af, bf[2], bf[3]);
+        }
+        const int h0 = mh * 16 + g;
+        if (!s_warp) {  // hand dP over
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int c = nk * 16 + 8 * j + 2 * tig;
+            *reinterpret_cast<float2*>(dpx + h0 * kDQP + c) = make_float2(acc2[j][0], acc2[j][1]);
+            *reinterpret_cast<float2*>(dpx + (h0 + 8) * kDQP + c) =
+                make_float2(acc2[j][2], acc2[j][3]);
           }
         }
-        {
-          const int h0 = wm * 16 + g, c0 = wn * 8 + 2 * tig;
-          float dsv[4];
+        __syncthreads();
+        if (s_warp) {  // dS = P (dP - delta) -> shared memory
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int head = h0 + ((q & 2) ? 8 : 0), key = c0 + (q & 1);
-            const float pr = key < n ? expf(sc[q] * scale - lse_s[head]) : 0.f;
-            dsv[q] = pr * (dp[q] - del_s[head]);
+          for (int j = 0; j < 2; ++j) {
+            const int c0 = nk * 16 + 8 * j + 2 * tig;
+            const float2 dlo = *reinterpret_cast<const float2*>(dpx + h0 * kDQP + c0);
+            const float2 dhi = *reinterpret_cast<const float2*>(dpx + (h0 + 8) * kDQP + c0);
+            const float dpv[4] = {dlo.x, dlo.y, dhi.x, dhi.y};
+            float dsv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int head = h0 + ((q & 2) ? 8 : 0), key = c0 + (q & 1);
+              const float pr = key < n ? expf(acc2[j][q] * scale - lse_s[head]) : 0.f;
+              dsv[q] = pr * (dpv[q] - del_s[head]);
+            }
+            *reinterpret_cast<uint32_t*>(Sd + h0 * kDS + c0) = pack_bf16(dsv[0], dsv[1]);
+            *reinterpret_cast<uint32_t*>(Sd + (h0 + 8) * kDS + c0) = pack_bf16(dsv[2], dsv[3]);
           }
-          *reinterpret_cast<uint32_t*>(Sd + h0 * kDS + c0) = pack_bf16(dsv[0], dsv[1]);
-          *reinterpret_cast<uint32_t*>(Sd + (h0 + 8) * kDS + c0) = pack_bf16(dsv[2], dsv[3]);
         }
         __syncthreads();
 #pragma unroll
