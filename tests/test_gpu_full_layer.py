@@ -150,3 +150,26 @@ def test_packed_workload_sampled():
                             device=DEV, doc_lengths=wl.docs())
     rows = synth.sample_rows(inp.cu_seqlens.cpu(), 8, 0)
     run_full(inp, wl.block_size, rows=rows, topk=wl.topk)
+
+
+@pytest.mark.slow
+def test_long_context_workload_sampled():
+    """T = 65536 in one document: 1024 key blocks per row, the per-SM block
+    scratch at its largest."""
+    wl = workloads.LONG
+    inp = synth.make_inputs(wl.total_tokens, wl.num_heads, wl.dk, wl.dv, dtype=wl.dtype, seed=0,
+                            device=DEV, doc_lengths=wl.docs())
+    rows = synth.sample_rows(inp.cu_seqlens.cpu(), 10, 0)
+    run_full(inp, wl.block_size, rows=rows, topk=wl.topk, want_blse=False)
+
+
+def test_short_workspace_is_refused():
+    inp = _inputs([300], 64, 576, 512, torch.bfloat16, seed=7)
+    need = hs.workspace_size(hs.HS_OP_BLOCK_SCORE_ATTN, 300, 1, inp.max_seqlen, 64, 576, 512,
+                             torch.bfloat16, 64)
+    assert need > 1024  # the fused kernel alone needs 2 x NBmax x 64 fp32 per SM
+    ws = torch.empty(1024, device=DEV, dtype=torch.uint8)
+    with pytest.raises(hs.HSError) as e:
+        hs.hs_block_score_attn_fwd(inp.q, inp.k, inp.v, inp.cu_seqlens, inp.max_seqlen, 64,
+                                   workspace=ws)
+    assert e.value.status == hs.HS_ERR_WORKSPACE

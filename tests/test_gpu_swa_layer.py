@@ -133,3 +133,22 @@ def test_main_workload_sampled():
     L = Layer(wl.docs(), wl.num_heads, wl.dk, wl.dv, wl.dtype, seed=0)
     rows = synth.sample_rows(L.cu.cpu(), 24, 0)
     run_layer(L, wl.block_size, wl.topk, wl.window, rows=rows)
+
+
+@pytest.mark.slow
+def test_packed_workload_sampled():
+    wl = workloads.PACKED
+    L = Layer(wl.docs(), wl.num_heads, wl.dk, wl.dv, wl.dtype, seed=0)
+    rows = synth.sample_rows(L.cu.cpu(), 6, 0)
+    run_layer(L, wl.block_size, wl.topk, wl.window, rows=rows)
+
+
+def test_empty_input_and_rejections():
+    L = Layer([64], 64, 576, 512, torch.bfloat16, seed=8)
+    idx = torch.zeros((64, 4), device=DEV, dtype=torch.int32)
+    with pytest.raises(hs.HSError) as e:  # window < 1
+        hs.hs_swa_layer_fwd(L.q, L.k, L.v, L.ks, L.vs, idx, L.cu, L.max_seqlen, 0, 64)
+    assert e.value.status == hs.HS_ERR_INVALID_ARG
+    with pytest.raises(ValueError):  # gates of the wrong shape
+        hs.hs_swa_layer_fwd(L.q, L.k, L.v, L.ks, L.vs, idx, L.cu, L.max_seqlen, 16, 64,
+                            gate_swa=torch.ones((64, 63), device=DEV))
