@@ -6,7 +6,7 @@
 // bq(t) of t's document, blockLSE = log sum_{j in block b, j <= t} exp(s_j),
 // LSE = log sum_{j <= t} exp(s_j), score[t, b] = sum_h exp(blockLSE - LSE).
 //
-// Design (one persistent CTA per SM, 6 warps):
+// Design (one persistent CTA per SM, 12 warps):
 //  * A query tile is 128 rows = (128 / H) consecutive tokens x H heads of one
 //    document; q[T, H, Dk] rows are (token, head) pairs, so a tile is a
 //    plain 128-row slab.  The first min(Dk, 512) columns of the tile live in
@@ -16,13 +16,15 @@
 //    RoPE part of Dk = 576) stays a shared-memory tile (SS form).
 //  * Keys stream in tiles of 128 (always a whole number of blocks, starting
 //    at the document's first token) as 64-column K chunks (one 16 KB TMA box
-//    each); three chunks form one 48 KB stage of a 4-deep ring, so every
-//    pipeline wait of the MMA thread is followed by 12 M=128, N=128, K=16
-//    MMAs issued without a branch between them (a wait costs a few hundred
-//    cycles of issue and a branch between two MMAs about half the issue
-//    rate; both were measured).  The shared-memory (RoPE) chunk goes first.
-//    Each key tile accumulates into one of two S buffers in TMEM (double
-//    buffering lets the MMA run one key tile ahead of the softmax).
+//    each); three chunks form one 48 KB stage, so every pipeline wait of an
+//    MMA thread is followed by 12 M=128, N=128, K=16 MMAs issued without a
+//    branch between them (a branch between two MMAs costs about half the
+//    issue rate).  The shared-memory (RoPE) chunk goes first.  Key tiles
+//    alternate between two MMA-issuing threads, each with its own producer
+//    and two-slot ring and its own S buffer in TMEM: a wait costs one issuing
+//    thread a few hundred cycles (measured: the stage waits took ~650 of the
+//    ~3800 cycles of a key tile with one issuer), and with two the tensor
+//    pipe runs the other thread's MMAs meanwhile.
 //  * Softmax warps (thread = row) read S (tcgen05.ld), compute per-block
 //    log-sum-exp in the log2 domain with the block's own max (no underflow
 //    for far-below-max blocks) and keep the running row max and sum.  Block
@@ -30,9 +32,11 @@
 //    L2 resident; halves alternate by query tile).  At the end of the tile each row has its LSE; the head
 //    sum of exp2(blockLSE - LSE) is a 32-lane transpose-reduction per warp
 //    plus a fixed-order sum over the warps of a token (deterministic).
-//  * Warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner), warps 2-9
-//    = two softmax warpgroups that take alternate S tiles (one S buffer
-//    each) and share the epilogue.  Per-row running
+//  * Warps 0 / 10 = TMA producers of rings 0 / 1 (warp 0 also loads q),
+//    warps 1 / 11 = MMA issuers of key tiles of even / odd index (warp 1 also
+//    copies q into TMEM and owns TMEM), warps 2-9 = two softmax warpgroups
+//    that take the alternate S tiles (one S buffer each) and share the
+//    epilogue.  Per-row running
 //    (max, sum) pairs of the two warpgroups are merged at the end of the
 //    tile; S is read in 32-column chunks with the next tcgen05.ld in flight.
 //    Every wait is bounded; a timeout records HS_ERR_TIMEOUT, drains
@@ -50,12 +54,15 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 320;  // producer, MMA, 2 softmax warpgroups
+constexpr int kThreads = 384;  // 2 producers, 2 MMA issuers, 2 softmax warpgroups
+constexpr int kProdB = 10;     // producer of ring 1
+constexpr int kMmaB = 11;      // MMA issuer of ring 1
 constexpr int kKeyTile = 128;
 constexpr int kChunkBytes = kKeyTile * 64 * 2;   // one TMA box: 128 keys x 64 bf16
 constexpr int kChunksPerStage = 3;               // 12 MMAs per pipeline wait
 constexpr int kStageBytes = kChunksPerStage * kChunkBytes;
-constexpr int kStages = 4;
+constexpr int kSlots = 2;                        // slots per ring (two rings)
+constexpr int kStages = 2 * kSlots;
 constexpr int kMaxQhi = 1;                       // shared-memory Q chunks (Dk <= 576)
 constexpr int kMaxTmemQ = 8;                     // TMEM Q chunks (first 512 columns)
 constexpr int kMaxDocs = 1024;
@@ -80,7 +87,10 @@ struct BSParams {
 
 struct Shared {
   uint64_t kfull[kStages], kempty[kStages];
-  uint64_t qhi_full, qhi_empty, qdone, drain;  // qdone: a tile's MMAs have completed
+  uint64_t qhi_full, qhi_empty;  // the shared-memory q chunk (empty: both issuers)
+  uint64_t qdone;                // a query tile's MMAs of both issuers have completed
+  uint64_t qready;               // issuer 0's copies of q into TMEM have completed
+  uint64_t drain[2];
   uint64_t sfull[2], sempty[2];
   uint64_t epi_all;    // rendezvous of both softmax warpgroups (256 threads)
   uint64_t epi_wg[2];  // rendezvous inside one warpgroup (128 threads)
@@ -181,9 +191,11 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
       mbar_init(&sh->kempty[s], 1);
     }
     mbar_init(&sh->qhi_full, 1);
-    mbar_init(&sh->qhi_empty, 1);
-    mbar_init(&sh->qdone, 1);
-    mbar_init(&sh->drain, 1);
+    mbar_init(&sh->qhi_empty, 2);
+    mbar_init(&sh->qdone, 2);
+    mbar_init(&sh->qready, 1);
+    mbar_init(&sh->drain[0], 1);
+    mbar_init(&sh->drain[1], 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->sfull[b], 1);
       mbar_init(&sh->sempty[b], 128);
@@ -215,90 +227,111 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
   const int G = gridDim.x, cta = blockIdx.x;
   const long long lim = p.wait_ns;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == kProdB) {
+    // ------------------------------------------------------------ producers
+    // Producer r fills ring r with the stages of the key tiles whose global
+    // index (key tiles counted over this CTA's query tiles) has parity r;
+    // producer 0 also loads each query tile's q: the shared-memory chunk and,
+    // through ring 0, the chunks that go to TMEM.
+    const int r = warp == 0 ? 0 : 1;
     if (lane == 0) {
       tma_prefetch_desc(&kmap);
-      tma_prefetch_desc(&qmap);
-      int fills[kStages];
+      if (r == 0) tma_prefetch_desc(&qmap);
+      int fills[kSlots];
 #pragma unroll
-      for (int s = 0; s < kStages; ++s) fills[s] = 0;
-      int qfills = 0;
+      for (int s2 = 0; s2 < kSlots; ++s2) fills[s2] = 0;
+      int qfills = 0, sbase = 0;
       uint32_t kst = 0, kph = 0;
-      for (int it = 0; it * G < total && !aborted(sh); ++it) {
+      bool stop = false;
+      // next stage of ring r: wait for the slot, arm its barrier
+      auto open_stage = [&](int bytes) -> uint8_t* {
+        const int sl = r * kSlots + (int)kst;
+        if (!mbar_wait(&sh->kempty[sl], kph ^ 1, lim)) return nullptr;
+        mbar_expect_tx(&sh->kfull[sl], bytes);
+        return stages + sl * kStageBytes;
+      };
+      auto close_stage = [&]() {
+        ++fills[kst];
+        if (++kst == kSlots) {
+          kst = 0;
+          kph ^= 1;
+        }
+      };
+      for (int it = 0; it * G < total && !stop && !aborted(sh); ++it) {
         const int g = it * G + ((it & 1) ? (G - 1 - cta) : cta);
         if (g >= total) continue;
         const Tile tl = tile_of(g, sh->prefix, nd, p.cu, p.tpt);
-        // warm L2 with the next tile's q rows (the softmax warps read them)
-        {
-          const int it2 = it + 1, g2 = it2 * G + ((it2 & 1) ? (G - 1 - cta) : cta);
-          if (g2 < total) {
-            const Tile t2 = tile_of(g2, sh->prefix, nd, p.cu, p.tpt);
-            for (int ch = 0; ch < p.nck; ++ch) tma_prefetch_3d(&qmap, ch * 64, 0, t2.t0);
-          }
-        }
-        if (p.nq_smem > 0) {
-          if (qfills > 0 && !mbar_wait(&sh->qhi_empty, (qfills - 1) & 1, lim)) {
-            give_up(sh, p.status);
-            break;
-          }
-          mbar_expect_tx(&sh->qhi_full, p.nq_smem * kChunkBytes);
-          for (int j = 0; j < p.nq_smem; ++j)
-            tma_load_3d(qhi + j * kChunkBytes, &qmap, &sh->qhi_full, (p.nq_tmem + j) * 64, 0,
-                        tl.t0);
-          ++qfills;
-        }
-        // the tile's q chunks that live in TMEM pass through the ring (three
-        // per stage); the MMA thread copies them into TMEM with tcgen05.cp
-        for (int q0 = 0; q0 < p.nq_tmem && !aborted(sh); q0 += kChunksPerStage) {
-          const int n = min(kChunksPerStage, p.nq_tmem - q0);
-          if (!mbar_wait(&sh->kempty[kst], kph ^ 1, lim)) {
-            give_up(sh, p.status);
-            break;
-          }
-          mbar_expect_tx(&sh->kfull[kst], n * kChunkBytes);
-          for (int j = 0; j < n; ++j)
-            tma_load_3d(stages + kst * kStageBytes + j * kChunkBytes, &qmap, &sh->kfull[kst],
-                        (q0 + j) * 64, 0, tl.t0);
-          ++fills[kst];
-          if (++kst == kStages) {
-            kst = 0;
-            kph ^= 1;
-          }
-        }
-        // per key tile, ring stages of three K chunks in the MMA's order: the
-        // shared-memory (RoPE) chunks first, then the TMEM chunks 0, 1, ...
         const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
-        const int spt = (p.nck + kChunksPerStage - 1) / kChunksPerStage;  // stages per key tile
-        for (int kt = 0; kt < nkt && !aborted(sh); ++kt) {
-          for (int st = 0; st < spt; ++st) {
-            const int nst = min(kChunksPerStage, p.nck - st * kChunksPerStage);
-            if (!mbar_wait(&sh->kempty[kst], kph ^ 1, lim)) {
-              give_up(sh, p.status);
+        if (r == 0) {
+          // warm L2 with the next tile's q rows (the softmax warps read them)
+          {
+            const int it2 = it + 1, g2 = it2 * G + ((it2 & 1) ? (G - 1 - cta) : cta);
+            if (g2 < total) {
+              const Tile t2 = tile_of(g2, sh->prefix, nd, p.cu, p.tpt);
+              for (int ch = 0; ch < p.nck; ++ch) tma_prefetch_3d(&qmap, ch * 64, 0, t2.t0);
+            }
+          }
+          if (p.nq_smem > 0) {
+            if (qfills > 0 && !mbar_wait(&sh->qhi_empty, (qfills - 1) & 1, lim)) {
+              stop = true;
               break;
             }
-            mbar_expect_tx(&sh->kfull[kst], nst * kChunkBytes);
+            mbar_expect_tx(&sh->qhi_full, p.nq_smem * kChunkBytes);
+            for (int j = 0; j < p.nq_smem; ++j)
+              tma_load_3d(qhi + j * kChunkBytes, &qmap, &sh->qhi_full, (p.nq_tmem + j) * 64, 0,
+                          tl.t0);
+            ++qfills;
+          }
+          // the tile's q chunks that live in TMEM pass through ring 0 (three
+          // per stage); MMA issuer 0 copies them into TMEM with tcgen05.cp
+          for (int q0 = 0; q0 < p.nq_tmem; q0 += kChunksPerStage) {
+            const int n = min(kChunksPerStage, p.nq_tmem - q0);
+            uint8_t* dst = open_stage(n * kChunkBytes);
+            if (!dst) { stop = true; break; }
+            const int sl = r * kSlots + (int)kst;
+            for (int j = 0; j < n; ++j)
+              tma_load_3d(dst + j * kChunkBytes, &qmap, &sh->kfull[sl], (q0 + j) * 64, 0, tl.t0);
+            close_stage();
+          }
+          if (stop) break;
+        }
+        // this ring's key tiles: stages of three K chunks in the MMA's order,
+        // the shared-memory (RoPE) chunks first, then the TMEM chunks 0, 1, ...
+        const int spt = (p.nck + kChunksPerStage - 1) / kChunksPerStage;  // stages per key tile
+        for (int kt = 0; kt < nkt && !stop; ++kt) {
+          if (((sbase + kt) & 1) != r) continue;
+          for (int st = 0; st < spt; ++st) {
+            const int nst = min(kChunksPerStage, p.nck - st * kChunksPerStage);
+            uint8_t* dst = open_stage(nst * kChunkBytes);
+            if (!dst) { stop = true; break; }
+            const int sl = r * kSlots + (int)kst;
             for (int j = 0; j < nst; ++j) {
               const int pos = st * kChunksPerStage + j;
               const int ch = pos < p.nq_smem ? p.nq_tmem + pos : pos - p.nq_smem;
-              tma_load_2d(stages + kst * kStageBytes + j * kChunkBytes, &kmap, &sh->kfull[kst],
-                          ch * 64, tl.bos + kt * kKeyTile);
+              tma_load_2d(dst + j * kChunkBytes, &kmap, &sh->kfull[sl], ch * 64,
+                          tl.bos + kt * kKeyTile);
             }
-            ++fills[kst];
-            if (++kst == kStages) {
-              kst = 0;
-              kph ^= 1;
-            }
+            close_stage();
           }
         }
+        sbase += nkt;
       }
+      if (stop) give_up(sh, p.status);
       // no copy may still be landing when the CTA exits
-      for (int s = 0; s < kStages; ++s)
-        if (fills[s] > 0) mbar_wait(&sh->kfull[s], (fills[s] - 1) & 1, kDefaultWaitNs);
+      for (int s2 = 0; s2 < kSlots; ++s2)
+        if (fills[s2] > 0)
+          mbar_wait(&sh->kfull[r * kSlots + s2], (fills[s2] - 1) & 1, kDefaultWaitNs);
       if (qfills > 0) mbar_wait(&sh->qhi_full, (qfills - 1) & 1, kDefaultWaitNs);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == kMmaB) {
+    // ------------------------------------------------------------ MMA issuers
+    // Issuer r issues the key tiles of global parity r from ring r into S
+    // buffer r (the softmax warpgroup r reads it); two instruction streams,
+    // so each one's pipeline waits overlap the other's MMAs.  Issuer 0 also
+    // copies each query tile's q into TMEM, once both issuers' MMAs of the
+    // previous tile are complete (qdone counts both), and commits qready,
+    // which issuer 1 waits for before its first MMA of the tile.
+    const int r = warp == 1 ? 0 : 1;
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
       uint64_t qhi_desc[kMaxQhi];
@@ -306,56 +339,74 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
       for (int j = 0; j < kMaxQhi; ++j)
         qhi_desc[j] = umma_desc_sw128(smem_u32(qhi + j * kChunkBytes), 16, 1024);
       const uint64_t stage_desc0 = umma_desc_sw128(smem_u32(stages), 16, 1024);
-      uint32_t kst = 0, kph = 0, sidx = 0;
-      int qtile = 0;
-      bool issued = false;
-      for (int it = 0; it * G < total && !aborted(sh); ++it) {
+      uint32_t kst = 0, kph = 0, myidx = 0;
+      int qtile = 0, sbase = 0;
+      bool issued = false, ok = true;
+      auto next_slot = [&]() {
+        if (++kst == kSlots) {
+          kst = 0;
+          kph ^= 1;
+        }
+      };
+      for (int it = 0; it * G < total && ok && !aborted(sh); ++it) {
         const int g = it * G + ((it & 1) ? (G - 1 - cta) : cta);
         if (g >= total) continue;
         const Tile tl = tile_of(g, sh->prefix, nd, p.cu, p.tpt);
         const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
-        // q enters TMEM by tcgen05.cp from the ring, once every MMA of the
-        // previous tile (which read the old q) has completed
-        if ((qtile > 0 && !mbar_wait_spin(&sh->qdone, (qtile - 1) & 1, lim)) ||
-            (p.nq_smem > 0 && !mbar_wait(&sh->qhi_full, qtile & 1, lim))) {
-          give_up(sh, p.status);
-          break;
-        }
-        tc_fence_after();
-        bool ok = true;
-        for (int q0 = 0; q0 < p.nq_tmem; q0 += kChunksPerStage) {
-          const int n = min(kChunksPerStage, p.nq_tmem - q0);
-          if (!mbar_wait_spin(&sh->kfull[kst], kph, lim)) {  // TMA stage
-            ok = false;
-            break;
-          }
-          const uint64_t b0 = stage_desc0 + (uint64_t)((kst * kStageBytes) >> 4);
-          for (int j = 0; j < n; ++j)
-#pragma unroll
-            for (int k = 0; k < 4; ++k)  // 128 rows x 16 elements per copy
-              tmem_cp_128x256b(tmem + (uint32_t)((q0 + j) * 32 + k * 8),
-                               b0 + (uint64_t)((j * kChunkBytes) >> 4) + 2 * k);
-          umma_commit(&sh->kempty[kst]);  // the copies have read the stage
-          if (++kst == kStages) {
-            kst = 0;
-            kph ^= 1;
-          }
-        }
-        const int spt = (p.nck + kChunksPerStage - 1) / kChunksPerStage;
-        for (int kt = 0; kt < nkt && ok; ++kt) {
-          const uint32_t buf = sidx & 1, use = sidx >> 1;
-          if (!mbar_wait_spin(&sh->sempty[buf], (use & 1) ^ 1, lim)) {
+        if (r == 0) {
+          // q enters TMEM by tcgen05.cp from the ring, once every MMA of the
+          // previous tile (which read the old q) has completed
+          if ((qtile > 0 && !mbar_wait_spin(&sh->qdone, (qtile - 1) & 1, lim)) ||
+              (p.nq_smem > 0 && !mbar_wait(&sh->qhi_full, qtile & 1, lim))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t d = tmem + kSCol + buf * 128;
-          for (int st = 0; st < spt; ++st) {
-            if (!mbar_wait_spin(&sh->kfull[kst], kph, lim)) {  // TMA stage (no fence needed)
+          for (int q0 = 0; q0 < p.nq_tmem; q0 += kChunksPerStage) {
+            const int n = min(kChunksPerStage, p.nq_tmem - q0);
+            const int sl = r * kSlots + (int)kst;
+            if (!mbar_wait_spin(&sh->kfull[sl], kph, lim)) {  // TMA stage
               ok = false;
               break;
             }
-            const uint64_t b0 = stage_desc0 + (uint64_t)((kst * kStageBytes) >> 4);
+            const uint64_t b0 = stage_desc0 + (uint64_t)((sl * kStageBytes) >> 4);
+            for (int j = 0; j < n; ++j)
+#pragma unroll
+              for (int k = 0; k < 4; ++k)  // 128 rows x 16 elements per copy
+                tmem_cp_128x256b(tmem + (uint32_t)((q0 + j) * 32 + k * 8),
+                                 b0 + (uint64_t)((j * kChunkBytes) >> 4) + 2 * k);
+            umma_commit(&sh->kempty[sl]);  // the copies have read the stage
+            next_slot();
+          }
+          if (!ok) break;
+          umma_commit(&sh->qready);  // arrives once the copies have completed
+          issued = true;
+        } else {
+          // every tile's phases, even with no key tile of this parity: a
+          // parity wait must never run two phases ahead of its barrier
+          if (!mbar_wait_spin(&sh->qready, qtile & 1, lim) ||
+              (p.nq_smem > 0 && !mbar_wait(&sh->qhi_full, qtile & 1, lim))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const int spt = (p.nck + kChunksPerStage - 1) / kChunksPerStage;
+        for (int kt = 0; kt < nkt && ok; ++kt) {
+          if (((sbase + kt) & 1) != r) continue;
+          if (!mbar_wait_spin(&sh->sempty[r], (myidx & 1) ^ 1, lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + kSCol + r * 128;
+          for (int st = 0; st < spt; ++st) {
+            const int sl = r * kSlots + (int)kst;
+            if (!mbar_wait_spin(&sh->kfull[sl], kph, lim)) {  // TMA stage (no fence needed)
+              ok = false;
+              break;
+            }
+            const uint64_t b0 = stage_desc0 + (uint64_t)((sl * kStageBytes) >> 4);
             // 12 MMAs without a branch between them (a branch between two
             // tcgen05.mma costs about half the issue rate); one stage pattern
             // is chosen per stage
@@ -376,27 +427,24 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
               else issue_stage<false, false, 1>(d, tmem, tpos, 0, b0, idesc);
             }
             issued = true;
-            umma_commit(&sh->kempty[kst]);
-            if (++kst == kStages) {
-              kst = 0;
-              kph ^= 1;
-            }
+            umma_commit(&sh->kempty[sl]);
+            next_slot();
           }
           if (!ok) break;
-          umma_commit(&sh->sfull[buf]);
-          ++sidx;
+          umma_commit(&sh->sfull[r]);
+          ++myidx;
         }
-        if (!ok) {
-          give_up(sh, p.status);
-          break;
-        }
+        if (!ok) break;
+        // this issuer is done with the tile's q (both commit; count 2)
         if (p.nq_smem > 0) umma_commit(&sh->qhi_empty);
         umma_commit(&sh->qdone);
         ++qtile;
+        sbase += nkt;
       }
-      if (issued) {  // every MMA done before TMEM is released
-        umma_commit(&sh->drain);
-        mbar_wait(&sh->drain, 0, kDefaultWaitNs);
+      if (!ok) give_up(sh, p.status);
+      if (issued) {  // every MMA and copy done before TMEM is released
+        umma_commit(&sh->drain[r]);
+        mbar_wait(&sh->drain[r], 0, kDefaultWaitNs);
       }
     }
   } else {

@@ -26,7 +26,7 @@ Sources (web pages, cited by title and section):
   the model-config section: a sparse pattern that covers every causal key is
   identical to dense causal attention.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * Block scoring carries no sink.  The block score of key block ``b`` for
   query ``t`` is the head-summed probability mass
