@@ -33,7 +33,9 @@
 // per head (raised only when a tile beats it by more than 2^8, which then
 // rescales O^T in TMEM), write P^T as bf16 into one 128-byte-swizzled buffer
 // and accumulate per-head sums in registers.  The sink joins in the
-// epilogue, which reads O^T back per dv row and writes out[t, h, :].
+// epilogue, which reads O^T back per dv row, stages each 128-row dv chunk
+// as [head][dv] in the P^T buffer and stores it to out[t, h, :] with one TMA
+// tensor store per warpgroup.
 // Warp 0 = K producer, warp 10 = V producer, warp 1 = QK issuer / TMEM
 // owner, warp 11 = PV issuer, warps 2-9 = two softmax warpgroups, each
 // owning 32 of the 64 heads (per-head state never crosses warpgroups).  All
@@ -258,7 +260,8 @@ template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap,
-                    const __grid_constant__ CUtensorMap qmap, const AttnParams p) {
+                    const __grid_constant__ CUtensorMap qmap,
+                    const __grid_constant__ CUtensorMap omap, const AttnParams p) {
   constexpr bool kSparse = kMode == kModeSparse;
   constexpr bool kFull = kMode == kModeFull;
   constexpr bool kCombine = kMode == kModeSwaLayer;
@@ -711,9 +714,12 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
       // O^T chunk c (dv rows x this warpgroup's 32 heads) is normalised,
       // staged as [head][128 dv] bf16 in this warpgroup's half of the P^T
-      // buffer (free: the token's last PV is complete) and written out as
-      // 16-byte stores, a head's 256 contiguous bytes per half-warp.  No wait
-      // inside this loop can fail, so all 128 threads meet each named barrier.
+      // buffer (free: the token's last PV is complete) and written out by
+      // one TMA tensor store of that box (the combining mode instead adds the
+      // other branch and writes 16-byte units, a head's 256 contiguous bytes
+      // per half-warp).  The storing thread waits until TMA has read the box
+      // before the next chunk is staged.  No wait inside this loop can fail,
+      // so all 128 threads meet each named barrier.
       {
         __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(pbuf) + wg * (32 * 128);
         __nv_bfloat16* obase = p.out + ((int64_t)t * kH + hb) * dvs;
@@ -742,6 +748,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
           for (int k = 0; k < 32; ++k)
             stage[k * 128 + r] = __float2bfloat16_rn(__uint_as_float(w[k]) * ls[k]);
+          if (!kCombine) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           named_bar(1 + wg, 128);
           if (kCombine) {
             // the gated other branch joins in fp32
@@ -765,13 +772,16 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
               }
             }
           } else {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const int u = r + 128 * q4;  // 16-byte unit: head u / 16, dv 8 (u % 16)
-              const uint4 v = reinterpret_cast<const uint4*>(stage)[u];
-              const int col = c * 128 + (u & 15) * 8;
-              if (col < dvs)  // a last chunk half past Dv holds zero rows
-                *reinterpret_cast<uint4*>(obase + (int64_t)(u >> 4) * dvs + col) = v;
+            // one thread stores the staged [32 heads][128 dv] box with TMA
+            // (columns past Dv fall outside the tensor and are not written)
+            if (r == 0) {
+              asm volatile(
+                  "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+                  ::"l"(reinterpret_cast<uint64_t>(&omap)), "r"(smem_u32(stage)), "r"(c * 128),
+                  "r"(hb), "r"(t)
+                  : "memory");
+              asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+              asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
             }
           }
           named_bar(1 + wg, 128);
@@ -810,6 +820,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
     }
     if (!ok) give_up(sh, p.status);
+    if (!kCombine && r == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 
   tc_fence_before();
@@ -842,7 +853,7 @@ cudaError_t launch_mode(const AttnArgs& a, int mode, const FullArgs* fa, long lo
   const bool sparse = mode == kModeSparse;
   const Problem& p = a.p;
   const uint32_t rows = sparse ? (uint32_t)a.block_size : (uint32_t)kTile;
-  CUtensorMap kmap, vmap, qmap;
+  CUtensorMap kmap, vmap, qmap, omap;
   {
     const uint64_t dims[2] = {(uint64_t)p.dk, (uint64_t)p.total_tokens};
     const uint64_t strides[1] = {(uint64_t)p.k_row_stride * 2};
@@ -860,6 +871,12 @@ cudaError_t launch_mode(const AttnArgs& a, int mode, const FullArgs* fa, long lo
     const uint64_t strides[2] = {(uint64_t)p.q_head_stride * 2, (uint64_t)p.q_row_stride * 2};
     const uint32_t box[3] = {64, (uint32_t)kH, 1};
     if (!encode_bf16_map(&qmap, p.q, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)p.dv, (uint64_t)p.num_heads, (uint64_t)p.total_tokens};
+    const uint64_t strides[2] = {(uint64_t)p.dv * 2, (uint64_t)p.num_heads * p.dv * 2};
+    const uint32_t box[3] = {128, 32, 1};
+    if (!encode_bf16_map(&omap, a.out, 3, dims, strides, box, false)) return cudaErrorInvalidValue;
   }
   AttnParams ap;
   ap.cu = p.cu_seqlens;
@@ -895,7 +912,7 @@ cudaError_t launch_mode(const AttnArgs& a, int mode, const FullArgs* fa, long lo
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemBytes, s>>>(kmap, vmap, qmap, ap);
+  kern<<<grid, kThreads, kSmemBytes, s>>>(kmap, vmap, qmap, omap, ap);
   return cudaGetLastError();
 }
 
