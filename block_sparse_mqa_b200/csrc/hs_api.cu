@@ -126,7 +126,7 @@ hs_status report_error(hs_status st, const char* msg) { return fail(st, "%s", ms
 
 extern "C" {
 
-int hs_version(void) { return 100; }
+int hs_version(void) { return 200; }
 
 const char* hs_status_string(hs_status s) {
   switch (s) {
