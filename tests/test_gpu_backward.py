@@ -156,6 +156,11 @@ def test_backward_with_v_aliasing_k():
     for gpu, name in zip(g, ("dq", "dk", "dv", "dsink")):
         check_grad(gpu, ref[name], torch.bfloat16, "aliased " + name)
 
+@pytest.mark.parametrize("kind", ["sparse", "swa"])
+def test_backward_zero_length_documents(kind):
+    run_backward([0, 150, 0, 0, 97, 0], 64, 576, 512, torch.bfloat16, kind, seed=12)
+
+
 def test_backward_other_dims():
     # Dk != Dv, not multiples of 64; several head groups with a partial last one
     run_backward([120, 88], 20, 80, 48, torch.float32, "sparse", B=16, K=3, seed=4)

@@ -102,6 +102,11 @@ def test_shape_variants_fused(dk, dv):
     run_full(inp, 64)
 
 
+def test_zero_length_documents():
+    inp = _inputs([0, 130, 0, 0, 257, 0], 64, 576, 512, torch.bfloat16, seed=8)
+    run_full(inp, 64)
+
+
 def test_forced_cuda_cores_agree():
     inp = _inputs([150, 90], 64, 576, 512, torch.bfloat16, seed=4)
     a = run_full(inp, 64)

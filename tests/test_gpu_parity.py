@@ -195,6 +195,29 @@ def test_shape_variants_on_tensor_cores(dk, dv):
         assert _expect_path(op, inp, 64) == hs.HS_PATH_TCGEN05, (op, dk, dv)
     run_and_check(inp, 64, 4, 100)
 
+@pytest.mark.parametrize("dtype,H,dk,dv", [(torch.bfloat16, 64, 576, 512),
+                                          (torch.float32, 4, 64, 48)])
+def test_zero_length_documents(dtype, H, dk, dv):
+    """cu_seqlens may repeat an offset (an empty document, e.g. padding);
+    empty documents own no rows and no blocks, and block numbering restarts
+    at each non-empty document."""
+    docs = [0, 200, 0, 0, 133, 0]
+    inp = _gpu_inputs(sum(docs), H, dk, dv, dtype, docs, seed=15)
+    run_and_check(inp, 64 if H == 64 else 16, 4, 100)
+
+
+def test_topk_at_maximum_covers_every_block():
+    """topk = 256 (the largest accepted) selects every causal block of these
+    documents, so block-sparse attention is dense causal attention, which the
+    window kernel computes with a window longer than the documents (the
+    oracle's invariant, here between the two GPU kernels)."""
+    docs = [700, 90]
+    inp = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=16)
+    res = run_and_check(inp, 16, 256, 1000)
+    P.check_out(res["out"], P.np64(res["swa_out"]), "sparse (all blocks) vs window (all keys)")
+    P.check_lse(res["lse"], P.np64(res["swa_lse"]), "sparse vs window lse")
+
+
 def test_force_simt_agrees_with_default_path():
     docs = [333, 80]
     inp = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=7)

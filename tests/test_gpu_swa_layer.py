@@ -117,6 +117,11 @@ def test_shared_v_aliases_shared_k_and_no_sinks():
     run_layer(L, 64, 4, 64, sinks=False)
 
 
+def test_zero_length_documents():
+    L = Layer([0, 130, 0, 0, 257, 0], 64, 576, 512, torch.bfloat16, seed=9)
+    run_layer(L, 64, 4, 100)
+
+
 def test_forced_cuda_cores_agree():
     L = Layer([150, 90], 64, 576, 512, torch.bfloat16, seed=4)
     a = run_layer(L, 64, 4, 80)
