@@ -112,3 +112,42 @@ def sample_rows(cu_seqlens, per_doc: int, seed: int = 0) -> np.ndarray:
         rows.extend([bos, eos - 1])
         rows.extend(int(bos + p) for p in pick)
     return np.unique(np.asarray(rows, dtype=np.int64))
+
+
+def plant_block_order(inp: Inputs, block_size: int, gap: float = 3.0, seed: int = 0,
+                      scale: Optional[float] = None, alpha: float = 4.0):
+    """Structured copy of ``inp`` whose top-k choice is well separated.
+
+    Each document d gets a seeded random permutation ``perms[d]`` of its key
+    blocks (``numpy.random.default_rng(seed + 104729).permutation``, one draw
+    per document, in document order).  Feature 0 of every query row is set to
+    ``alpha`` and feature 0 of key j (doc-local block b of document d) to
+    ``gap * perms[d][b] / (scale * alpha)``, so that a logit
+    ``scale * <q, k_j>`` is the other features' random product plus
+    ``gap * perms[d][b]`` (up to the rounding of that one key value to the
+    input dtype).  With ``gap`` far above the spread of a block's random
+    log-mass, every head ranks the complete blocks of a document in
+    ``perms[d]`` order.  ``scale`` defaults to Dk^-1/2.  Returns
+    ``(inputs, perms)``; the caller's tensors are not modified.
+    """
+    dk = inp.q.shape[2]
+    sc = float(dk) ** -0.5 if scale is None else float(scale)
+    cu = [int(x) for x in inp.cu_seqlens.tolist()]
+    rng = np.random.default_rng(seed + 104729)
+    perms = []
+    val = np.zeros(inp.total_tokens, dtype=np.float64)
+    for bos, eos in zip(cu[:-1], cu[1:]):
+        nb = (eos - bos + block_size - 1) // block_size
+        perm = rng.permutation(nb) if nb > 0 else np.zeros(0, dtype=np.int64)
+        perms.append(perm)
+        for j in range(bos, eos):
+            val[j] = gap * float(perm[(j - bos) // block_size]) / (sc * alpha)
+    q = inp.q.clone()
+    k = inp.k.clone()
+    q[:, :, 0] = alpha
+    k[:, 0] = torch.as_tensor(val, dtype=torch.float32, device=k.device).to(k.dtype)
+    meta = dict(inp.meta)
+    meta.update({"planted_gap": gap, "planted_seed": seed, "planted_alpha": alpha})
+    return Inputs(q=q, k=k, v=inp.v, sink=inp.sink, cu_seqlens=inp.cu_seqlens,
+                  max_seqlen=inp.max_seqlen, meta=meta), perms
+

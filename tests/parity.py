@@ -98,3 +98,30 @@ def bq_rows(cu, rows, block_size):
         d = max(i for i in range(len(cu) - 1) if cu[i] <= t)
         out.append((int(t) - cu[d]) // block_size)
     return out
+
+
+def planted_selection(cu_seqlens, perms, block_size: int, topk: int, rows=None) -> np.ndarray:
+    """The selection that a planted block order (synth.plant_block_order)
+    implies, written from the selection rule of the pages (the query's own
+    block and block 0 forced, the rest by descending score) with the scores'
+    order taken from ``perms`` instead of computed: per query t of document d with own
+    block bq, every block 0..bq when bq + 1 <= topk, else blocks 0 and bq plus
+    the topk - 2 blocks of 1..bq-1 with the largest ``perms[d]`` (topk = 1:
+    the own block alone); ascending, padded with -1.  Rows default to every
+    token."""
+    cu = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    T = cu[-1]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    out = np.full((len(rows), topk), -1, dtype=np.int32)
+    for i, t in enumerate(rows):
+        d = max(x for x in range(len(cu) - 1) if cu[x] <= t < cu[x + 1])
+        bq = (int(t) - cu[d]) // block_size
+        if bq + 1 <= topk:
+            sel = list(range(bq + 1))
+        elif topk == 1:
+            sel = [bq]
+        else:
+            rest = sorted(range(1, bq), key=lambda b: -int(perms[d][b]))[:topk - 2]
+            sel = sorted({0, bq, *rest})
+        out[i, :len(sel)] = sel
+    return out

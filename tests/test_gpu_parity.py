@@ -218,6 +218,20 @@ def test_topk_at_maximum_covers_every_block():
     P.check_lse(res["lse"], P.np64(res["swa_lse"]), "sparse vs window lse")
 
 
+@pytest.mark.parametrize("B,K,docs", [(64, 6, [700, 0, 420]), (16, 10, [400, 0, 300])])
+def test_planted_block_order_selects_exactly(B, K, docs):
+    """Structured inputs (synth.plant_block_order, gap 3 natural-log units
+    per rank): the block order is planted, so the GPU's index sets must equal
+    the selection rule's choice for that order exactly, with no near-tie
+    excusal; every step still matches the oracle.  Documents stay under 27
+    blocks so that no selected block's fp32 score underflows."""
+    base = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=17)
+    inp, perms = synth.plant_block_order(base, B, gap=3.0, seed=17)
+    res = run_and_check(inp, B, K, 100)
+    expect = P.planted_selection(inp.cu_seqlens.cpu(), perms, B, K)
+    np.testing.assert_array_equal(res["idx"].cpu().numpy(), expect)
+
+
 def test_force_simt_agrees_with_default_path():
     docs = [333, 80]
     inp = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=7)

@@ -23,6 +23,7 @@ import torch
 import oracle.hysparse as O
 from oracle import loops
 from block_sparse_mqa_b200 import synth
+from tests import parity as P
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden", "closed_form.json")
 
@@ -345,6 +346,25 @@ def test_attention_matches_loops(with_sink):
                                       None if sink is None else sink.tolist(), sc)
     np.testing.assert_allclose(w["out"], out, rtol=1e-11, atol=1e-13)
     np.testing.assert_allclose(w["lse"], lse, rtol=1e-13)
+
+
+@pytest.mark.parametrize("K", [1, 2, 5, 8])
+def test_selection_follows_a_planted_block_order(K):
+    """Scores with a planted order (synth.plant_block_order: every logit of a
+    key in block b gains 3 * perm[b] natural-log units) must make the
+    oracle's step 1 + step 2 pick exactly the blocks that the selection rule
+    ("HySparse MQA sparse attention ..." pull request, hs_select_topk: own
+    block and block 0 forced, the rest by descending block score, ties to
+    the lower id) implies for that order, computed here without any scores.
+    A reversed sort, a dropped forced block or a wrong causal limit fails."""
+    base = synth.make_inputs(300, 4, 64, 48, dtype=torch.float32, seed=21,
+                             doc_lengths=[0, 170, 0, 130])
+    inp, perms = synth.plant_block_order(base, 16, gap=3.0, seed=21)
+    f = lambda t: t.double().numpy()
+    cu = inp.cu_seqlens.tolist()
+    bs = O.block_score(f(inp.q), f(inp.k), cu, 16)
+    idx = O.select_topk(bs["block_score"], cu, 16, K, total_tokens=300)
+    np.testing.assert_array_equal(idx, P.planted_selection(cu, perms, 16, K))
 
 
 def test_selection_structure():
