@@ -79,6 +79,10 @@ def ncu_traffic(kernel):
 
 
 NOMINAL_BF16_TFLOPS = 2250.0   # dense bf16, per GPU (context only)
+# a step at least this long keeps the GPU under sustained load (the clocks
+# settle under the power cap): its tensor kernels are measured against the
+# sustained bf16 peak, shorter steps against the burst peak
+LONG_STEP_MS = 20.0
 NOMINAL_HBM_GBS = 8000.0
 
 
@@ -428,10 +432,12 @@ def run_ours(args, wl, world, rank):
     nb = hs.nbmax(inp.max_seqlen, wl.block_size)
     sel_bytes = 4.0 * sum(((n - 1) // wl.block_size + 1) * n for n in wl.docs()) + 4.0 * wl.total_tokens * wl.topk
     avg = {ph: statistics.mean(per_phase[p]) for p, ph in enumerate(Step.PHASES)}
+    sustained = sum(avg.values()) >= LONG_STEP_MS and pk.get("bf16_tflops_sustained")
+    tpk = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
     kernels = {}
     for ph in ("score", "sparse", "swa"):
         tf = flops[ph] / (avg[ph] / 1e3) / 1e12
-        kernels[ph] = {"ms": avg[ph], "tflops": tf, "frac_of_bf16_peak": tf / pk["bf16_tflops"],
+        kernels[ph] = {"ms": avg[ph], "tflops": tf, "frac_of_bf16_peak": tf / tpk,
                        "frac_of_nominal_bf16": tf / NOMINAL_BF16_TFLOPS,
                        "algorithmic_flops": flops[ph],
                        "path": "tcgen05" if hs.path(
@@ -447,11 +453,12 @@ def run_ours(args, wl, world, rank):
                          "frac_of_nominal_hbm": sel_gbs / NOMINAL_HBM_GBS,
                          "algorithmic_bytes": sel_bytes, "path": "simt"}
     dom = max(("score", "sparse", "swa"), key=lambda ph: avg[ph])
-    roof = {"bound": "tensor", "achieved": kernels[dom]["tflops"], "peak": pk["bf16_tflops"],
-            "unit": "TFLOP/s", "frac": kernels[dom]["tflops"] / pk["bf16_tflops"],
+    roof = {"bound": "tensor", "achieved": kernels[dom]["tflops"], "peak": tpk,
+            "unit": "TFLOP/s", "frac": kernels[dom]["tflops"] / tpk,
             "traffic": ncu_traffic(dom) if wl.name == workloads.MAIN.name else None,
             "kernel": dom,
-            "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % pk["source"]}
+            "peak_source": "%s bf16 %s (MEASURED_PEAKS.json)" % (
+                pk["source"], "sustained: step >= %g ms" % LONG_STEP_MS if sustained else "burst")}
     contraction_tflops = (flops["score"] + flops["sparse"] + flops["swa"]) / (
         (avg["score"] + avg["sparse"] + avg["swa"]) / 1e3) / 1e12
 
