@@ -1,6 +1,7 @@
-// The dq and dk / dv passes of the attention backward on warp-level
-// tensor-core MMAs (mma.sync m16n8k16, bf16 in, fp32 accumulate), for bf16
-// inputs with 64 heads, Dk and Dv multiples of 64 (Dk <= 576, Dv <= 512).
+// The dk / dv pass of the attention backward on warp-level tensor-core MMAs
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate), for bf16 inputs with 64
+// heads, Dk and Dv multiples of 64 (Dk <= 576, Dv <= 512); the dq pass runs
+// on tcgen05 (tc_bwd_dq.cu).
 //
 // Definitions as in simt_backward.cu ("HySparse MQA sparse attention ...",
 // PaddleFleet pull request 1470, "Core" list: SWA and block-sparse MQA
@@ -401,180 +402,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_mma_kernel(const MmaBwdP
   }
 }
 
-// ---------------------------------------------------------------- dq
-// Query-major: one CTA per token t with q_t and dout_t (all heads) resident;
-// the token's key set in tiles of at most 32 keys that never cross a block
-// (SWA: the window).  Per tile:
-//   S [64 heads x 32 keys] = q_t . K_tile^T   (warps 0-7, 16 x 16 each)
-//   dP = dout_t . V_tile^T                    (warps 8-15, 16 x 16 each;
-//       handed to the S warps through an fp32 tile)
-//   dS = P (dP - delta) -> shared memory (bf16, [head][key])
-//   dQ [64 x Dk] += dS . K_tile   (registers: warp w owns heads 16 (w / 4)..
-//       and every fourth 8-column tile from w % 4)
-constexpr int kDS = kKT + kPad;  // row stride of the dS tile
-constexpr int kMaxNQ = 18;       // Dk / 32 n-tiles per warp (Dk <= 576)
-
-constexpr int kDQP = kKT + 8;    // fp32 row stride of the dP hand-over tile
-
-inline size_t mma_dq_smem_bytes(int dk, int dv) {
-  const int KS = dk + kPad, VS = dv + kPad;
-  return 2 * ((size_t)kH * KS + (size_t)kH * VS + (size_t)kKT * KS + (size_t)kKT * VS +
-              (size_t)kH * kDS) +
-         4 * (size_t)kH * kDQP + 4 * 2 * (size_t)kH + 4 * 256;
-}
-
-template <bool kSparse>
-__global__ void __launch_bounds__(kThreads, 1) bwd_dq_mma_kernel(const MmaBwdParams a) {
-  extern __shared__ __align__(16) uint8_t smraw[];
-  __shared__ int nblk;
-  const Problem& P = a.p;
-  const int dk = P.dk, dv = P.dv, KS = dk + kPad, VS = dv + kPad;
-  __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(smraw);  // [kH][KS]
-  __nv_bfloat16* Ds = Qs + kH * KS;                              // [kH][VS]
-  __nv_bfloat16* Kt = Ds + kH * VS;                              // [kKT][KS]
-  __nv_bfloat16* Vt = Kt + kKT * KS;                             // [kKT][VS]
-  __nv_bfloat16* Sd = Vt + kKT * VS;                             // [kH][kDS] dS
-  float* dpx = reinterpret_cast<float*>(Sd + kH * kDS);          // [kH][kDQP] dP
-  float* lse_s = dpx + kH * kDQP;
-  float* del_s = lse_s + kH;
-  int* blist = reinterpret_cast<int*>(del_s + kH);               // [256]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, tig = lane & 3;
-  const int wm = warp >> 2;  // 16-head tile
-  const int wn = warp & 3;   // 8-key tile (scores) / n-tile phase (dq)
-  const int nQ = dk >> 5;
-  const float scale = P.scale;
-  const uint32_t kt_base = (uint32_t)__cvta_generic_to_shared(Kt);
-  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(P.q);
-  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(P.k);
-  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(P.v);
-  // Score phase: warp w < 8 computes S, warp w + 8 dP at the same place:
-  // heads 16 mh.., keys 16 nk.. (two n8 tiles sharing each A fragment).
-  const bool s_warp = warp < 8;
-  const int mh = (warp >> 1) & 3, nk = warp & 1;
-  const uint32_t a_sc = (uint32_t)__cvta_generic_to_shared(s_warp ? Qs : Ds) +
-                        (uint32_t)(((mh * 16 + (lane & 15)) * (s_warp ? KS : VS) +
-                                    (lane >> 4) * 8) * 2);
-  const uint32_t b_sc = (uint32_t)__cvta_generic_to_shared(s_warp ? Kt : Vt) +
-                        (uint32_t)(((nk * 16 + (lane & 7) + ((lane >> 4) << 3)) *
-                                        (s_warp ? KS : VS) +
-                                    ((lane >> 3) & 1) * 8) * 2);
-  const int kend_sc = s_warp ? dk : dv;
-  for (int t = blockIdx.x; t < P.total_tokens; t += gridDim.x) {
-    int bos, eos;
-    if (!find_doc(P.cu_seqlens, P.num_docs, P.total_tokens, P.max_seqlen, t, bos, eos, P.status))
-      continue;
-    if (kSparse && tid == 0) {
-      const int bq = (t - bos) / a.B;
-      const int32_t* row = a.idx + (int64_t)t * a.topk;
-      int nb = 0;
-      bool bad = false;
-      for (int sl = 0; sl < a.topk; ++sl) {
-        int b;
-        if (entry_used(row, sl, bq, b)) blist[nb++] = b;
-        else if (b >= 0) bad = true;
-      }
-      if (bad) record_status(P.status, HS_ERR_INVALID_INDEX);
-      nblk = nb;
-    }
-    stage_token(Qs, KS, Ds, VS, qg, P.q_row_stride, P.q_head_stride, a.dout, t, dk, dv);
-    if (tid < kH) {
-      lse_s[tid] = __ldg(a.lse + (int64_t)t * kH + tid);
-      del_s[tid] = __ldg(a.delta + (int64_t)t * kH + tid);
-    }
-    cp_async_wait_all();
-    float acc[kMaxNQ][4];
-#pragma unroll
-    for (int i = 0; i < kMaxNQ; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    __syncthreads();
-    const int nseg = kSparse ? nblk : 1;
-    for (int sg = 0; sg < nseg; ++sg) {
-      int lo, hi;
-      if (kSparse) {
-        lo = bos + blist[sg] * a.B;
-        hi = min(min(lo + a.B, eos), t + 1);
-      } else {
-        lo = max(bos, t - a.window + 1);
-        hi = t + 1;
-      }
-      for (int j0 = lo; j0 < hi; j0 += kKT) {
-        const int n = min(kKT, hi - j0);
-        copy_rows(Kt, KS, kg + (int64_t)j0 * P.k_row_stride, P.k_row_stride, n, dk, kKT);
-        copy_rows(Vt, VS, vg + (int64_t)j0 * P.v_row_stride, P.v_row_stride, n, dv, kKT);
-        cp_async_wait_all();
-        __syncthreads();
-        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        for (int k0 = 0; k0 < kend_sc; k0 += 16) {
-          uint32_t af[4], bf[4];
-          ldsm_x4(af, a_sc + (uint32_t)(k0 * 2));
-          ldsm_x4(bf, b_sc + (uint32_t)(k0 * 2));
-          mma16816(acc2[0], af, bf[0], bf[1]);
-          mma16816(acc2[1], af, bf[2], bf[3]);
-        }
-        const int h0 = mh * 16 + g;
-        if (!s_warp) {  // hand dP over
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int c = nk * 16 + 8 * j + 2 * tig;
-            *reinterpret_cast<float2*>(dpx + h0 * kDQP + c) = make_float2(acc2[j][0], acc2[j][1]);
-            *reinterpret_cast<float2*>(dpx + (h0 + 8) * kDQP + c) =
-                make_float2(acc2[j][2], acc2[j][3]);
-          }
-        }
-        __syncthreads();
-        if (s_warp) {  // dS = P (dP - delta) -> shared memory
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int c0 = nk * 16 + 8 * j + 2 * tig;
-            const float2 dlo = *reinterpret_cast<const float2*>(dpx + h0 * kDQP + c0);
-            const float2 dhi = *reinterpret_cast<const float2*>(dpx + (h0 + 8) * kDQP + c0);
-            const float dpv[4] = {dlo.x, dlo.y, dhi.x, dhi.y};
-            float dsv[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int head = h0 + ((q & 2) ? 8 : 0), key = c0 + (q & 1);
-              const float pr = key < n ? expf(acc2[j][q] * scale - lse_s[head]) : 0.f;
-              dsv[q] = pr * (dpv[q] - del_s[head]);
-            }
-            *reinterpret_cast<uint32_t*>(Sd + h0 * kDS + c0) = pack_bf16(dsv[0], dsv[1]);
-            *reinterpret_cast<uint32_t*>(Sd + (h0 + 8) * kDS + c0) = pack_bf16(dsv[2], dsv[3]);
-          }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int ks = 0; ks < kKT / 16; ++ks) {
-          const __nv_bfloat16* sa = Sd + (wm * 16 + g) * kDS + ks * 16 + 2 * tig;
-          const uint32_t af[4] = {lds32(sa), lds32(sa + 8 * kDS), lds32(sa + 8),
-                                  lds32(sa + 8 * kDS + 8)};
-          const uint32_t krow = kt_base + (uint32_t)((ks * 16 + (lane & 15)) * KS) * 2u;
-#pragma unroll
-          for (int i = 0; i < kMaxNQ; ++i) {
-            if (i < nQ) {
-              uint32_t b0, b1;
-              ldsm_x2_trans(b0, b1, krow + (uint32_t)((wn + 4 * i) * 16));
-              mma16816(acc[i], af, b0, b1);
-            }
-          }
-        }
-        __syncthreads();
-      }
-    }
-    {
-      const int h0 = wm * 16 + g;
-      float* dq0 = a.dq + ((int64_t)t * kH + h0) * dk;
-#pragma unroll
-      for (int i = 0; i < kMaxNQ; ++i) {
-        if (i < nQ) {
-          const int col = (wn + 4 * i) * 8 + 2 * tig;
-          *reinterpret_cast<float2*>(dq0 + col) = make_float2(scale * acc[i][0], scale * acc[i][1]);
-          *reinterpret_cast<float2*>(dq0 + 8 * dk + col) =
-              make_float2(scale * acc[i][2], scale * acc[i][3]);
-        }
-      }
-    }
-    __syncthreads();
-  }
-}
-
 }  // namespace
 
 bool mma_backward_shape_ok(hs_dtype dtype, int num_heads, int dk, int dv) {
@@ -587,28 +414,7 @@ bool mma_backward_supported(const Problem& p) {
   return mma_backward_shape_ok(p.dtype, p.num_heads, p.dk, p.dv) &&
          al16(p.q) && al16(p.k) && al16(p.v) && p.q_row_stride % 8 == 0 &&
          p.q_head_stride % 8 == 0 && p.k_row_stride % 8 == 0 && p.v_row_stride % 8 == 0 &&
-         mma_dkdv_smem_bytes(p.dk, p.dv) <= 227 * 1024 && mma_dq_smem_bytes(p.dk, p.dv) <= 227 * 1024;
-}
-
-cudaError_t launch_mma_dq(const BwdArgs& b, bool sparse, const float* delta, cudaStream_t s) {
-  MmaBwdParams a;
-  a.p = b.p;
-  a.idx = b.idx;
-  a.topk = b.topk;
-  a.B = b.block_size;
-  a.window = b.window;
-  a.lse = b.lse;
-  a.delta = delta;
-  a.dout = static_cast<const __nv_bfloat16*>(b.dout);
-  a.dkey = nullptr;
-  a.dval = nullptr;
-  a.dq = b.dq;
-  const size_t bytes = mma_dq_smem_bytes(b.p.dk, b.p.dv);
-  auto kern = sparse ? bwd_dq_mma_kernel<true> : bwd_dq_mma_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e != cudaSuccess) return e;
-  kern<<<b.p.total_tokens, kThreads, bytes, s>>>(a);
-  return cudaGetLastError();
+         mma_dkdv_smem_bytes(p.dk, p.dv) <= 227 * 1024;
 }
 
 cudaError_t launch_mma_dkdv(const BwdArgs& b, bool sparse, const float* delta, cudaStream_t s) {

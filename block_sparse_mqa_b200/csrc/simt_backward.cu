@@ -467,11 +467,14 @@ cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, bool allow_mma, 
   a.delta = static_cast<float*>(b.workspace);
   a.dsink_part = a.delta + (size_t)b.p.total_tokens * b.p.num_heads;
   if (b.p.dtype == HS_BF16) {
-    const bool mma = allow_mma && mma_backward_supported(b.p);
+    // tensor cores: dq on tcgen05, dk / dv on warp-level MMAs (else every
+    // pass on CUDA cores)
+    const bool mma = allow_mma && mma_backward_supported(b.p) && tc_bwd_dq_supported(b.p) &&
+                     (reinterpret_cast<uintptr_t>(b.dout) & 15) == 0;
     cudaError_t e = sparse ? launch_typed<__nv_bfloat16, true>(a, !mma, s)
                            : launch_typed<__nv_bfloat16, false>(a, !mma, s);
     if (e != cudaSuccess || !mma) return e;
-    e = launch_mma_dq(b, sparse, a.delta, s);
+    e = launch_tc_bwd_dq(b, sparse, a.delta, 0, s);
     if (e != cudaSuccess) return e;
     return launch_mma_dkdv(b, sparse, a.delta, s);
   }
