@@ -629,7 +629,7 @@ def run_backward(inp, wl, step, cu, pk, reps=2):
         tf = fl / (ms / 1e3) / 1e12
         res[name] = {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / pk["bf16_tflops"],
                      "algorithmic_flops": fl, "calls_timed": reps,
-                     "path": {hs.HS_PATH_MMA: "dq tcgen05, dk/dv mma.sync",
+                     "path": {hs.HS_PATH_MMA: "tcgen05",
                               hs.HS_PATH_SIMT: "simt"}.get(
                          hs.path(hs.HS_OP_SPARSE_MQA_BWD if name == "sparse" else hs.HS_OP_SWA_MQA_BWD,
                                  wl.dtype, H, wl.dk, wl.dv, wl.block_size), "other")}

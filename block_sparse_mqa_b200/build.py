@@ -64,7 +64,13 @@ def build(jobs: int = 8, verbose: bool = False) -> str:
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     with cf.ThreadPoolExecutor(max_workers=jobs) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
-    if os.path.exists(LIB) and os.path.getmtime(LIB) >= max(os.path.getmtime(o) for o in objs):
+    # relink when an object is newer than the library or the set of sources
+    # changed (a file added or removed)
+    manifest = os.path.join(BUILD, "link_inputs.txt")
+    listed = "\n".join(objs)
+    same_set = os.path.exists(manifest) and open(manifest).read() == listed
+    if (same_set and os.path.exists(LIB) and
+            os.path.getmtime(LIB) >= max(os.path.getmtime(o) for o in objs)):
         return LIB
     tmp = LIB + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcuda"]
@@ -73,6 +79,8 @@ def build(jobs: int = 8, verbose: bool = False) -> str:
         sys.stderr.write(res.stdout + res.stderr)
         raise RuntimeError("link failed")
     os.replace(tmp, LIB)
+    with open(manifest, "w") as f:
+        f.write(listed)
     return LIB
 
 

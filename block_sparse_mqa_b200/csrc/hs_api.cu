@@ -165,7 +165,7 @@ int hs_path(int op, hs_dtype dtype, int num_heads, int dk, int dv, int block_siz
       return HS_PATH_SIMT;
     case HS_OP_SPARSE_MQA_BWD:
     case HS_OP_SWA_MQA_BWD:
-      if (!g_force_simt.load() && hs::mma_backward_shape_ok(dtype, num_heads, dk, dv))
+      if (!g_force_simt.load() && hs::tc_backward_shape_ok(dtype, num_heads, dk, dv))
         return HS_PATH_MMA;
       return HS_PATH_SIMT;
     case HS_OP_SPARSE_MQA:

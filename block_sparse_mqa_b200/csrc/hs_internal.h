@@ -87,16 +87,17 @@ cudaError_t launch_select_topk(const float* block_score, int nb_stride, const in
 cudaError_t launch_simt_attention(const AttnArgs& a, bool sparse, cudaStream_t s);
 size_t simt_backward_workspace(int total_tokens, int num_heads);
 cudaError_t launch_simt_backward(const BwdArgs& a, bool sparse, bool allow_mma, cudaStream_t s);
-// key-major dk/dv pass on warp-level tensor-core MMAs (bf16, 64 heads, Dk
-// and Dv multiples of 64); delta = the workspace's [T, H] array.
-bool mma_backward_shape_ok(hs_dtype dtype, int num_heads, int dk, int dv);
-bool mma_backward_supported(const Problem& p);
-cudaError_t launch_mma_dkdv(const BwdArgs& a, bool sparse, const float* delta, cudaStream_t s);
-// dq on tcgen05 (bf16, 64 heads, Dk <= 576 and Dv <= 512, multiples of 64,
-// 16-byte aligned operands); delta as above
+// The backward's tcgen05 passes: bf16, 64 heads, Dk <= 576 and Dv <= 512,
+// multiples of 64, 16-byte aligned operands; delta = the workspace's [T, H]
+// array.  dq query-major (tc_bwd_dq.cu); dk / dv key-major, a cluster of
+// four CTAs per 32-key tile (tc_bwd_dkdv.cu).
+bool tc_backward_shape_ok(hs_dtype dtype, int num_heads, int dk, int dv);
 bool tc_bwd_dq_supported(const Problem& p);
+bool tc_bwd_dkdv_supported(const Problem& p);
 cudaError_t launch_tc_bwd_dq(const BwdArgs& a, bool sparse, const float* delta,
                              long long wait_limit, cudaStream_t s);
+cudaError_t launch_tc_bwd_dkdv(const BwdArgs& a, bool sparse, const float* delta,
+                               long long wait_limit, cudaStream_t s);
 
 // Shared-memory bytes the CUDA-core block-score kernel needs (0 if it cannot run).
 size_t simt_block_score_smem(int num_heads, int dk, int nbmax);

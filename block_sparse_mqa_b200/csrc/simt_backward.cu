@@ -467,16 +467,15 @@ cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, bool allow_mma, 
   a.delta = static_cast<float*>(b.workspace);
   a.dsink_part = a.delta + (size_t)b.p.total_tokens * b.p.num_heads;
   if (b.p.dtype == HS_BF16) {
-    // tensor cores: dq on tcgen05, dk / dv on warp-level MMAs (else every
-    // pass on CUDA cores)
-    const bool mma = allow_mma && mma_backward_supported(b.p) && tc_bwd_dq_supported(b.p) &&
+    // tensor cores: dq and dk / dv on tcgen05 (else every pass on CUDA cores)
+    const bool mma = allow_mma && tc_bwd_dq_supported(b.p) && tc_bwd_dkdv_supported(b.p) &&
                      (reinterpret_cast<uintptr_t>(b.dout) & 15) == 0;
     cudaError_t e = sparse ? launch_typed<__nv_bfloat16, true>(a, !mma, s)
                            : launch_typed<__nv_bfloat16, false>(a, !mma, s);
     if (e != cudaSuccess || !mma) return e;
     e = launch_tc_bwd_dq(b, sparse, a.delta, 0, s);
     if (e != cudaSuccess) return e;
-    return launch_mma_dkdv(b, sparse, a.delta, s);
+    return launch_tc_bwd_dkdv(b, sparse, a.delta, 0, s);
   }
   return sparse ? launch_typed<float, true>(a, true, s) : launch_typed<float, false>(a, true, s);
 }

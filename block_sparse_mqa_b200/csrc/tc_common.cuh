@@ -222,6 +222,20 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr, uint32_t
   return d;
 }
 
+// MN-major operand with 64-byte swizzle (layout type 4): each K row holds 32
+// contiguous MN elements (64 B); 8 K rows form a 512-B group, the next group
+// follows at SBO; chunk bits 4-5 of an address are XOR-ed with bits 7-8.
+__device__ __forceinline__ uint64_t umma_desc_sw64(uint32_t smem_addr, uint32_t lbo_bytes,
+                                                   uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFF) >> 4);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version (sm_100)
+  d |= (uint64_t)4 << 61;  // 64-byte swizzle
+  return d;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulate.
 // c_format F32 (bit 4), a_format/b_format BF16 (bits 7 and 10), a/b major
 // (bits 15/16: 0 = K-major, 1 = MN-major), N >> 3 in [17,23), M >> 4 in

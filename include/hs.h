@@ -109,9 +109,8 @@ typedef enum hs_op {
 typedef enum hs_kernel_path {
   HS_PATH_SIMT = 0,    /* CUDA-core kernel: fp32 inputs, unusual shapes    */
   HS_PATH_TCGEN05 = 1, /* tcgen05 tensor-core kernel (TMEM accumulators)   */
-  HS_PATH_MMA = 2      /* the backward's tensor-core path: dq on tcgen05,
-                          dk / dv on warp-level MMAs (register accumulators:
-                          a key tile's dk / dv exceed TMEM)                */
+  HS_PATH_MMA = 2      /* the backward's tensor-core path (tcgen05: a
+                          query-major dq pass and a key-major dk / dv pass) */
 } hs_kernel_path;
 
 /*
@@ -252,10 +251,10 @@ hs_status hs_swa_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_str
  * idx entries follow the forward's rule; offending entries are skipped and
  * reported as HS_ERR_INVALID_INDEX.  Results are deterministic (every sum
  * runs in a fixed order).  bf16 inputs with 64 heads and Dk, Dv multiples of
- * 64 (Dk <= 576, Dv <= 512, 16-byte aligned) run on tensor cores (hs_path:
- * HS_PATH_MMA): dq on tcgen05, dk / dv on warp-level MMAs; other inputs on
- * CUDA cores.  The dk / dv pass is a four-CTA cluster kernel that falls back
- * to single CTAs where the device cannot place the cluster.
+ * 64 (Dk <= 576, Dv <= 512, 16-byte aligned) run on tcgen05 tensor cores
+ * (hs_path: HS_PATH_MMA); other inputs on CUDA cores.  The dk / dv pass is a
+ * four-CTA cluster kernel that falls back to single CTAs where the device
+ * cannot place the cluster.
  */
 hs_status hs_sparse_mqa_bwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
                             const void* k, int64_t k_row_stride,
