@@ -110,11 +110,11 @@ def test_backward_block_and_window_variants(B, K, W):
 @pytest.mark.parametrize("B,K,W,dk,dv", [(16, 3, 1, 128, 64), (32, 2, 700, 192, 128),
                                          (128, 5, 129, 512, 448), (64, 4, 64, 64, 512)])
 def test_backward_tensor_core_variants(B, K, W, dk, dv):
-    """64 heads in bf16 take the tensor-core passes (tcgen05 dq over 128-key
-    tiles, warp-level key-major dk/dv over 32-key tiles): block sizes whose
-    blocks a 32-key tile can straddle (three at B = 16), documents that start
-    off the tile grids, Dk / Dv multiples of 64 down to a single 64-column
-    chunk and a ragged last 128-column stage (Dv = 448)."""
+    """64 heads in bf16 take the tcgen05 passes (query-major dq over 128-key
+    tiles, key-major dk/dv over 32-key tiles): block sizes whose blocks a
+    32-key tile can straddle (three at B = 16), documents that start off the
+    tile grids, Dk / Dv multiples of 64 down to a single 64-column chunk and
+    a ragged last 128-row chunk (Dv = 448)."""
     docs = [300, 37, 180]
     for kind in ("sparse", "swa"):
         run_backward(docs, 64, dk, dv, torch.bfloat16, kind, B=B, K=K, W=W, seed=3)
