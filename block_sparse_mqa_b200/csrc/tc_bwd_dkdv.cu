@@ -73,8 +73,9 @@ struct DkdvParams {
 };
 
 struct Shared {
-  uint64_t tile_full, qfull, dfull, qfree, dfree, sdp_full, sdp_empty, pds_full, pds_free,
-      acc_done;
+  uint64_t tile_full, sdp_full, sdp_empty, pds_full, pds_free, acc_done;
+  // per 64-column chunk of q_t / dout_t: loaded, and read by the member's MMAs
+  uint64_t qfull[kMaxQC], qfree[kMaxQC], dfull[kMaxDC], dfree[kMaxDC];
   int mem[kThreads];      // a candidate chunk's members (query tokens)
   int memmask[kThreads];  // and the tile keys each attends (bit jj = key s0 + jj)
   int wcount[kThreads / 32];
@@ -145,10 +146,14 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap kmap,
 
   if (tid == 0) {
     mbar_init(&sh->tile_full, 1);
-    mbar_init(&sh->qfull, 1);
-    mbar_init(&sh->dfull, 1);
-    mbar_init(&sh->qfree, 1);
-    mbar_init(&sh->dfree, 1);
+    for (int c = 0; c < kMaxQC; ++c) {
+      mbar_init(&sh->qfull[c], 1);
+      mbar_init(&sh->qfree[c], 1);
+    }
+    for (int c = 0; c < kMaxDC; ++c) {
+      mbar_init(&sh->dfull[c], 1);
+      mbar_init(&sh->dfree[c], 1);
+    }
     mbar_init(&sh->sdp_full, 2);   // both issuers' commits
     mbar_init(&sh->sdp_empty, 128);
     mbar_init(&sh->pds_full, 128);
@@ -241,28 +246,28 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap kmap,
         __syncthreads();
         // ---- this CTA's members of the chunk (every csize-th, ascending)
         if (warp == 0) {
-          // producer: q_t and dout_t of each member, once the previous
-          // member's MMAs have read the buffers
+          // producer: q_t and dout_t of each member, chunk c by lane c, each
+          // chunk once the previous member's MMAs have read it (the next
+          // member's loads overlap this member's last MMAs)
           uint32_t m = nmem;
           for (int mi = crank; mi < nm && ok; mi += csize, ++m) {
             const int tt = sh->mem[mi];
             int good = 1;
-            if (lane == 0) {
-              if (m > 0) good = mbar_wait(&sh->qfree, (m - 1) & 1, lim);
-              if (good) mbar_expect_tx(&sh->qfull, (uint32_t)p.nck * kTokChunk);
+            if (lane < p.nck) {
+              if (m > 0) good = mbar_wait(&sh->qfree[lane], (m - 1) & 1, lim);
+              if (good) {
+                mbar_expect_tx(&sh->qfull[lane], kTokChunk);
+                tma_load_3d(qb + lane * kTokChunk, &qmap, &sh->qfull[lane], lane * 64, 0, tt);
+              }
             }
-            good = __shfl_sync(0xffffffffu, good, 0);
-            if (!good) { ok = false; break; }
-            __syncwarp();
-            if (lane < p.nck) tma_load_3d(qb + lane * kTokChunk, &qmap, &sh->qfull, lane * 64, 0, tt);
-            if (lane == 0) {
-              if (m > 0) good = mbar_wait(&sh->dfree, (m - 1) & 1, lim);
-              if (good) mbar_expect_tx(&sh->dfull, (uint32_t)p.ndc * kTokChunk);
+            if (good && lane < p.ndc) {
+              if (m > 0) good = mbar_wait(&sh->dfree[lane], (m - 1) & 1, lim);
+              if (good) {
+                mbar_expect_tx(&sh->dfull[lane], kTokChunk);
+                tma_load_3d(db + lane * kTokChunk, &dmap, &sh->dfull[lane], lane * 64, 0, tt);
+              }
             }
-            good = __shfl_sync(0xffffffffu, good, 0);
-            if (!good) { ok = false; break; }
-            __syncwarp();
-            if (lane < p.ndc) tma_load_3d(db + lane * kTokChunk, &dmap, &sh->dfull, lane * 64, 0, tt);
+            if (!__all_sync(0xffffffffu, good)) { ok = false; break; }
           }
         } else if (warp == 1 || warp == 2) {
           // two MMA-issuing threads: warp 1 issues the q side (S, then dK^T),
@@ -278,8 +283,8 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap kmap,
             const int nmc = qside ? nmk : nmv;
             const uint32_t col_s = qside ? kColS : kColDP;
             const uint32_t col_acc = qside ? kColDK : kColDV;
-            uint64_t* const full_b = qside ? &sh->qfull : &sh->dfull;
-            uint64_t* const free_b = qside ? &sh->qfree : &sh->dfree;
+            uint64_t* const full_b = qside ? sh->qfull : sh->dfull;
+            uint64_t* const free_b = qside ? sh->qfree : sh->dfree;
             uint32_t m = nmem;
             for (int mi = crank; mi < nm && ok; mi += csize, ++m) {
               if (!tile_waited) {
@@ -287,31 +292,38 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap kmap,
                 tile_waited = true;
               }
               // S (or dP) of this member, once the previous member's were read
-              if ((m > 0 && !mbar_wait_spin(&sh->sdp_empty, (m - 1) & 1, lim)) ||
-                  !mbar_wait_spin(full_b, m & 1, lim)) {
+              if (m > 0 && !mbar_wait_spin(&sh->sdp_empty, (m - 1) & 1, lim)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
-              for (int c = 0; c < nch; ++c)
+              bool got = true;
+              for (int c = 0; c < nch && got; ++c) {
+                if (!mbar_wait_spin(&full_b[c], m & 1, lim)) { got = false; break; }
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                   umma_ss(tmem + col_s, a_k + (uint64_t)((c * kTokChunk) >> 4) + 2 * k,
                           b_k + (uint64_t)((c * kRowChunk) >> 4) + 2 * k, id_s,
                           (c == 0 && k == 0) ? 0u : 1u);
+              }
+              if (!got) { ok = false; break; }
               umma_commit(&sh->sdp_full);
               // dK^T += q_t^T . dS (or dV^T += dout_t^T . P) once P and dS are
               // written (the tile's first member opens the sums)
               if (!mbar_wait_spin(&sh->pds_full, m & 1, lim)) { ok = false; break; }
               tc_fence_after();
               const uint32_t first = any ? 1u : 0u;
-              for (int c = 0; c < nmc; ++c)
+              for (int c = 0; c < nmc; ++c) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                   umma_ss(tmem + col_acc + c * kKT,
                           a_mn + (uint64_t)((2 * c * kTokChunk) >> 4) + (uint64_t)(k * 128),
                           b_pd + (uint64_t)(k * 64), id_acc, (k == 0) ? first : 1u);
-              umma_commit(free_b);
+                // this chunk pair of q_t (or dout_t) is read: the next member's
+                // copies may land there
+                umma_commit(&free_b[2 * c]);
+                if (2 * c + 1 < nch) umma_commit(&free_b[2 * c + 1]);
+              }
               umma_commit(&sh->pds_free);
               any = true;
             }
@@ -440,11 +452,9 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap kmap,
     }
   }
   // every TMA copy issued has landed before the CTA exits
-  if (warp == 0 && lane == 0) {
-    if (nmem > 0) {
-      mbar_wait(&sh->qfull, (nmem - 1) & 1, kDefaultWaitNs);
-      mbar_wait(&sh->dfull, (nmem - 1) & 1, kDefaultWaitNs);
-    }
+  if (warp == 0 && nmem > 0) {
+    if (lane < p.nck) mbar_wait(&sh->qfull[lane], (nmem - 1) & 1, kDefaultWaitNs);
+    if (lane < p.ndc) mbar_wait(&sh->dfull[lane], (nmem - 1) & 1, kDefaultWaitNs);
   }
   tc_fence_before();
   __syncthreads();
