@@ -26,8 +26,10 @@
 // member in ascending order, and the four partial sums are added in rank
 // order through distributed shared memory, so a tile every query selects (a
 // document's first block) is spread over four SMs.  Per member the producer
-// loads q_t and dout_t by TMA into their buffers once the previous member's
-// MMAs have read them.  Sums run in a fixed order: results are deterministic.
+// loads q_t and dout_t by TMA chunk by chunk, each 64-column chunk once the
+// previous member's dK^T / dV^T MMAs have read it, and two threads issue the
+// MMAs (the q side and the dout side).  Sums run in a fixed order: results
+// are deterministic.
 // All waits are bounded (HS_ERR_TIMEOUT).
 
 #include <cooperative_groups.h>
