@@ -58,8 +58,12 @@ def parse():
                     help="skip the (separately timed) full layer's fused forward")
     ap.add_argument("--no-swa-layer", action="store_true",
                     help="skip the (separately timed) combined SWA layer")
-    ap.add_argument("--cpu-rows", type=int, default=3072,
-                    help="query rows of the oracle sample (cpu_baseline / reference arm)")
+    ap.add_argument("--cpu-rows", type=int, default=4096,
+                    help="query rows of the oracle sample (cpu_baseline / reference arm); "
+                         "4096 covers the main workload whole")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-setting timings of the packed, long-context and "
+                         "sweep workloads")
     return ap.parse_args()
 
 
@@ -283,10 +287,12 @@ def run_cpu_baseline(wl, rows_n, steps=1):
         oracle_step(O, host, rows, wl)
     dt = time.perf_counter() - t0
     used, aff, blas = cpu_cores()
+    what = ("all %d query rows of %s (the whole workload)" % (len(rows), wl.name)
+            if len(rows) == wl.total_tokens else "%d query rows of %s" % (len(rows), wl.name))
     return {"value": len(rows) * steps / dt, "unit": UNIT, "cores": used, "kind": "oracle",
-            "sample": "%d query rows of %s (all four steps, float64 NumPy), %d step(s), %.1f s; "
+            "sample": "%s, all four steps, float64 NumPy, %d step(s), %.1f s; "
                       "os.cpu_count() %d, affinity %d cores, BLAS threads %d" % (
-                          len(rows), wl.name, steps, dt, os.cpu_count() or 0, aff, blas)}
+                          what, steps, dt, os.cpu_count() or 0, aff, blas)}
 
 
 # ---------------------------------------------------------------------------
@@ -475,6 +481,10 @@ def run_ours(args, wl, world, rank):
     if not args.no_swa_layer:
         layer = run_swa_layer(inp, wl, step, pk, flush, flops["sparse"] + flops["swa"],
                               avg["sparse"] + avg["swa"])
+    other = None
+    if not args.no_workloads and world == 1 and wl.name == workloads.MAIN.name:
+        torch.cuda.empty_cache()
+        other = run_workloads(pk, flush)
 
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -496,7 +506,123 @@ def run_ours(args, wl, world, rank):
         "backward": bwd,
         "full_layer": full,
         "swa_layer": layer,
+        "workloads": other,
     }
+    return res
+
+
+def _timed(fn, flush, reps, warm=2):
+    """CUDA-event milliseconds of fn() per call (mean of reps), L2 flushed
+    before each call outside the events, after warm untimed calls."""
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for r in range(reps):
+        flush.fill_(r & 0xff)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.mean(ts)
+
+
+def run_workloads(pk, flush, reps=3):
+    """Per-setting numbers of the other workloads: the packed 16384-token
+    one, the 65536-token long context, the 4 x 32768 sparsity sweep (top-k 8,
+    16, 32, 64; block scoring depends on no top-k, so it is timed once for
+    the four) and the sweep's separate SWA-only layer (Dk 192 / Dv 128,
+    windows 256, 1024, 4096).  Each kernel: CUDA-event time per call (mean of
+    `reps`, L2 flushed before each, two untimed calls first), its
+    algorithmic work and the fraction of the bf16 peak; a step of 20 ms or
+    more is measured against the sustained peak, shorter ones against the
+    burst peak.  SM clocks are sampled during each workload's timed calls."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    res = {}
+
+    def frac_of(ms_total):
+        sus = ms_total >= LONG_STEP_MS and pk.get("bf16_tflops_sustained")
+        return (pk["bf16_tflops_sustained"] if sus else pk["bf16_tflops"]), \
+            ("sustained" if sus else "burst")
+
+    def kern(ms, fl, peak):
+        tf = fl / (ms / 1e3) / 1e12
+        return {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / peak, "algorithmic_flops": fl}
+
+    def one(wl, topks, with_swa=True, swa_only=False):
+        inp = synth.make_inputs(wl.total_tokens, wl.num_heads, wl.dk, wl.dv, dtype=wl.dtype,
+                                seed=0, device=dev, doc_lengths=wl.docs())
+        cu = inp.cu_seqlens.cpu().tolist()
+        H, T = wl.num_heads, wl.total_tokens
+        clocks = ClockSampler(dev.index)
+        clocks.start()
+        out = {}
+        if swa_only:
+            o = torch.empty((T, H, wl.dv), device=dev, dtype=wl.dtype)
+            l = torch.empty((T, H), device=dev, dtype=torch.float32)
+            ms = _timed(lambda: hs.hs_swa_mqa_fwd(inp.q, inp.k, inp.v, inp.cu_seqlens,
+                                                  inp.max_seqlen, wl.window, inp.sink, out=o,
+                                                  lse=l), flush, reps)
+            peak, kind = frac_of(ms)
+            out = {"swa": kern(ms, 2.0 * H * (wl.dk + wl.dv) * window_pairs(wl.docs(), wl.window),
+                               peak),
+                   "tokens_per_s": T / (ms / 1e3), "peak": kind}
+        else:
+            step = Step(inp, wl)
+            ms_score = _timed(step.score, flush, reps)
+            per_k = {}
+            for k in topks:
+                w2 = workloads.Workload(wl.name, T, H, wl.dk, wl.dv, wl.dtype, wl.block_size, k,
+                                        wl.window, wl.doc_lengths)
+                st = Step(inp, w2)
+                st.bs, st.ws, st.lse1 = step.bs, step.ws, step.lse1
+                ms_sel = _timed(st.select, flush, reps)
+                ms_sp = _timed(st.sparse, flush, reps)
+                ms_tot = ms_score + ms_sel + ms_sp
+                peak, kind = frac_of(ms_tot)
+                pairs = sparse_pairs(st.idx, cu, wl.block_size)
+                sel_bytes = 4.0 * sum(((n - 1) // wl.block_size + 1) * n for n in wl.docs() if n) \
+                    + 4.0 * T * k
+                per_k[k] = {
+                    "score": kern(ms_score, 2.0 * H * wl.dk * causal_pairs(wl.docs()), peak),
+                    "select": {"ms": ms_sel, "gbs": sel_bytes / (ms_sel / 1e3) / 1e9,
+                               "frac_of_hbm": sel_bytes / (ms_sel / 1e3) / 1e9 / pk["hbm_gbs"],
+                               "algorithmic_bytes": sel_bytes},
+                    "sparse": kern(ms_sp, 2.0 * H * (wl.dk + wl.dv) * pairs, peak),
+                    "score_select_sparse_tokens_per_s": T / (ms_tot / 1e3), "peak": kind}
+                del st
+            if with_swa:
+                ms_swa = _timed(step.swa, flush, reps)
+                k0 = topks[0]
+                peak = pk["bf16_tflops_sustained"] if per_k[k0]["peak"] == "sustained" \
+                    else pk["bf16_tflops"]
+                per_k[k0]["swa"] = kern(ms_swa, 2.0 * H * (wl.dk + wl.dv) *
+                                        window_pairs(wl.docs(), wl.window), peak)
+                tot = ms_score + per_k[k0]["select"]["ms"] + per_k[k0]["sparse"]["ms"] + ms_swa
+                per_k[k0]["step_tokens_per_s"] = T / (tot / 1e3)
+            out = per_k[topks[0]] if len(topks) == 1 else {"topk_%d" % k: v for k, v in per_k.items()}
+            del step
+        out["clocks"] = clocks.stop()
+        out["config"] = {"tokens": T, "docs": len(wl.docs()), "num_heads": H, "dk": wl.dk,
+                         "dv": wl.dv, "block_size": wl.block_size, "window": wl.window}
+        del inp
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        return out
+
+    t0 = time.perf_counter()
+    res[workloads.PACKED.name] = one(workloads.PACKED, [workloads.PACKED.topk])
+    res[workloads.LONG.name] = one(workloads.LONG, [workloads.LONG.topk])
+    sw = workloads.sweep(16)
+    res["sweep_4x32768_H64_dk576_dv512_bf16_B64"] = one(sw, [8, 16, 32, 64], with_swa=False)
+    for w in (256, 1024, 4096):
+        wl = workloads.sweep_swa(w)
+        res[wl.name] = one(wl, [], swa_only=True)
+    hs.poll_status(dev)
+    res["wall_s"] = time.perf_counter() - t0
     return res
 
 

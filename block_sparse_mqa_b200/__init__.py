@@ -8,4 +8,4 @@ B200 (sm_100a).
 * ``build``     compiles libhs.so in-tree for sm_100a.
 """
 
-__version__ = "0.1.0"
+__version__ = "0.3.0"  # = hs_version() of libhs.so (major.minor.patch)

@@ -28,6 +28,9 @@ std::atomic<int> g_force_simt{0};
 std::atomic<long long> g_wait_limit{0};  // 0 = the kernels' default bound
 
 thread_local char g_last_error[512];
+// Kernel family of the calling thread's most recent successful compute call
+// (hs_last_path), -1 before the first one.
+thread_local int g_last_path = -1;
 
 hs_status fail(hs_status st, const char* fmt, ...) {
   va_list ap;
@@ -116,17 +119,42 @@ hs_status launched(cudaError_t e, const char* what) {
   return HS_OK;
 }
 
+// launched(), and on success records `path` as the call's kernel family.
+hs_status launched_on(cudaError_t e, const char* what, int path) {
+  hs_status r = launched(e, what);
+  if (r == HS_OK) g_last_path = path;
+  return r;
+}
+
 }  // namespace
 
 namespace hs {
 // Lets other translation units of the library report a host-side failure
 // through hs_last_error().
 hs_status report_error(hs_status st, const char* msg) { return fail(st, "%s", msg); }
+
+// Host checks of hs_block_score's arguments, without any device work.
+hs_status check_score_args(const void* q, int64_t qrs, int64_t qhs, const void* k, int64_t krs,
+                           const int32_t* cu, int num_docs, int total_tokens, int max_seqlen,
+                           int num_heads, int dk, hs_dtype dtype, float scale, int block_size,
+                           const float* lse, const float* block_score, int nb_stride) {
+  Problem p{};
+  hs_status r = check_problem(p, q, qrs, qhs, k, krs, cu, num_docs, total_tokens, max_seqlen,
+                              num_heads, dk, 0, dtype, scale);
+  if (r != HS_OK) return r;
+  if (!valid_block(block_size))
+    return fail(HS_ERR_UNSUPPORTED, "block_size %d not in {16, 32, 64, 128}", block_size);
+  if (!lse || !block_score) return fail(HS_ERR_INVALID_ARG, "lse or block_score is NULL");
+  if (total_tokens > 0 && nb_stride < nbmax_of(max_seqlen, block_size))
+    return fail(HS_ERR_INVALID_ARG, "nb_stride %d < ceil(max_seqlen / block_size) = %d", nb_stride,
+                nbmax_of(max_seqlen, block_size));
+  return HS_OK;
+}
 }  // namespace hs
 
 extern "C" {
 
-int hs_version(void) { return 200; }
+int hs_version(void) { return 300; }
 
 const char* hs_status_string(hs_status s) {
   switch (s) {
@@ -142,6 +170,8 @@ const char* hs_status_string(hs_status s) {
 }
 
 const char* hs_last_error(void) { return g_last_error; }
+
+int hs_last_path(void) { return g_last_path; }
 
 void hs_set_force_simt(int on) { g_force_simt.store(on ? 1 : 0); }
 
@@ -258,14 +288,15 @@ hs_status hs_block_score(const void* q, int64_t q_row_stride, int64_t q_head_str
     if (need > 0 && (!workspace || workspace_bytes < need))
       return fail(HS_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
                   workspace ? workspace_bytes : (size_t)0);
-    return launched(hs::launch_tc_block_score(a, g_wait_limit.load(), stream), "tc block score");
+    return launched_on(hs::launch_tc_block_score(a, g_wait_limit.load(), stream),
+                       "tc block score", HS_PATH_TCGEN05);
   }
   int dev = 0, optin = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (hs::simt_block_score_smem(num_heads, dk, nbmax) > (size_t)optin)
     return fail(HS_ERR_UNSUPPORTED, "num_heads * dk + blocks too large for the CUDA-core kernel");
-  return launched(hs::launch_simt_block_score(a, stream), "simt block score");
+  return launched_on(hs::launch_simt_block_score(a, stream), "simt block score", HS_PATH_SIMT);
 }
 
 hs_status hs_select_topk(const float* block_score, int nb_stride, const int32_t* cu_seqlens,
@@ -283,13 +314,16 @@ hs_status hs_select_topk(const float* block_score, int nb_stride, const int32_t*
   if (nb_stride < nbmax)
     return fail(HS_ERR_INVALID_ARG, "nb_stride %d < ceil(max_seqlen / block_size) = %d", nb_stride,
                 nbmax);
+  if (nbmax > hs::kMaxSelectBlocks)
+    return fail(HS_ERR_UNSUPPORTED, "ceil(max_seqlen / block_size) = %d blocks > %d", nbmax,
+                hs::kMaxSelectBlocks);
   int* st = nullptr;
   hs_status r = status_ptr(&st);
   if (r != HS_OK) return r;
-  return launched(hs::launch_select_topk(block_score, nb_stride, cu_seqlens, num_docs,
-                                         total_tokens, max_seqlen, block_size, topk, idx, st,
-                                         stream),
-                  "select topk");
+  return launched_on(hs::launch_select_topk(block_score, nb_stride, cu_seqlens, num_docs,
+                                            total_tokens, max_seqlen, block_size, topk, idx, st,
+                                            stream),
+                     "select topk", HS_PATH_SIMT);
 }
 
 static hs_status attention_common(hs::AttnArgs& a, bool sparse, const void* q, int64_t qrs,
@@ -316,10 +350,11 @@ static hs_status attention_common(hs::AttnArgs& a, bool sparse, const void* q, i
   const bool tc = dtype == HS_BF16 && !g_force_simt.load() &&
                   hs::tc_attention_supported(num_heads, dk, dv, a.block_size, sparse) &&
                   hs::tc_attention_eligible(a);
-  if (tc) return launched(hs::launch_tc_attention(a, sparse, g_wait_limit.load(), stream),
-                          sparse ? "tc sparse attention" : "tc swa attention");
-  return launched(hs::launch_simt_attention(a, sparse, stream),
-                  sparse ? "simt sparse attention" : "simt swa attention");
+  if (tc) return launched_on(hs::launch_tc_attention(a, sparse, g_wait_limit.load(), stream),
+                             sparse ? "tc sparse attention" : "tc swa attention",
+                             HS_PATH_TCGEN05);
+  return launched_on(hs::launch_simt_attention(a, sparse, stream),
+                     sparse ? "simt sparse attention" : "simt swa attention", HS_PATH_SIMT);
 }
 
 hs_status hs_sparse_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
@@ -411,7 +446,8 @@ hs_status hs_block_score_attn_fwd(const void* q, int64_t q_row_stride, int64_t q
     if (!workspace || workspace_bytes < need)
       return fail(HS_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
                   workspace ? workspace_bytes : (size_t)0);
-    return launched(hs::launch_tc_full(f, g_wait_limit.load(), stream), "tc full layer");
+    return launched_on(hs::launch_tc_full(f, g_wait_limit.load(), stream), "tc full layer",
+                       HS_PATH_TCGEN05);
   }
   // two kernels: the attention (its lse is the same quantity; the score
   // kernel then writes lse again), then step 1
@@ -422,10 +458,11 @@ hs_status hs_block_score_attn_fwd(const void* q, int64_t q_row_stride, int64_t q
                    : hs::launch_simt_attention(a, false, stream),
                "full layer attention");
   if (r != HS_OK) return r;
-  return hs_block_score(q, q_row_stride, q_head_stride, k, k_row_stride, cu_seqlens, num_docs,
-                        total_tokens, max_seqlen, num_heads, dk, dtype, softmax_scale,
-                        block_size, lse, block_score, nb_stride, block_lse, workspace,
-                        workspace_bytes, stream);
+  r = hs_block_score(q, q_row_stride, q_head_stride, k, k_row_stride, cu_seqlens, num_docs,
+                     total_tokens, max_seqlen, num_heads, dk, dtype, softmax_scale, block_size,
+                     lse, block_score, nb_stride, block_lse, workspace, workspace_bytes, stream);
+  if (r == HS_OK && !tca) g_last_path = HS_PATH_SIMT;  // the attention ran on CUDA cores
+  return r;
 }
 
 hs_status hs_swa_layer_fwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
@@ -467,6 +504,7 @@ hs_status hs_swa_layer_fwd(const void* q, int64_t q_row_stride, int64_t q_head_s
                                  num_docs, total_tokens, max_seqlen, num_heads, dk, dv, dtype,
                                  softmax_scale, sink_sparse, out, lse_sparse, stream);
   if (r != HS_OK) return r;
+  const int sparse_path = g_last_path;
   // the window branch, whose epilogue adds the gated sparse result from out
   hs::AttnArgs w{};
   w.idx = nullptr;
@@ -476,9 +514,11 @@ hs_status hs_swa_layer_fwd(const void* q, int64_t q_row_stride, int64_t q_head_s
   w.prev = out;
   w.gate_own = gate_swa;
   w.gate_prev = gate_sparse;
-  return attention_common(w, false, q, q_row_stride, q_head_stride, k, k_row_stride, v,
-                          v_row_stride, cu_seqlens, num_docs, total_tokens, max_seqlen,
-                          num_heads, dk, dv, dtype, softmax_scale, sink_swa, out, lse_swa, stream);
+  r = attention_common(w, false, q, q_row_stride, q_head_stride, k, k_row_stride, v,
+                       v_row_stride, cu_seqlens, num_docs, total_tokens, max_seqlen, num_heads,
+                       dk, dv, dtype, softmax_scale, sink_swa, out, lse_swa, stream);
+  if (r == HS_OK && sparse_path == HS_PATH_SIMT) g_last_path = HS_PATH_SIMT;
+  return r;
 }
 
 static hs_status backward_common(hs::BwdArgs& a, bool sparse, const void* q, int64_t qrs,
@@ -517,8 +557,9 @@ static hs_status backward_common(hs::BwdArgs& a, bool sparse, const void* q, int
   a.workspace = workspace;
   r = status_ptr(&a.p.status);
   if (r != HS_OK) return r;
-  return launched(hs::launch_simt_backward(a, sparse, !g_force_simt.load(), stream),
-                  sparse ? "simt sparse attention backward" : "simt swa attention backward");
+  int path = HS_PATH_SIMT;
+  return launched_on(hs::launch_simt_backward(a, sparse, !g_force_simt.load(), &path, stream),
+                     sparse ? "sparse attention backward" : "swa attention backward", path);
 }
 
 hs_status hs_sparse_mqa_bwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,

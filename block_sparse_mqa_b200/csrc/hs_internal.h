@@ -81,12 +81,17 @@ struct BwdArgs {
 
 // Launchers; each returns cudaSuccess or the launch error.
 cudaError_t launch_simt_block_score(const ScoreArgs& a, cudaStream_t s);
+// Longest score row hs_select_topk takes (its keys staged in shared memory):
+// NBmax = ceil(max_seqlen / block_size) <= kMaxSelectBlocks.
+constexpr int kMaxSelectBlocks = 56 * 1024;
 cudaError_t launch_select_topk(const float* block_score, int nb_stride, const int32_t* cu,
                                int num_docs, int total_tokens, int max_seqlen, int block_size,
                                int topk, int32_t* idx, int* status, cudaStream_t s);
 cudaError_t launch_simt_attention(const AttnArgs& a, bool sparse, cudaStream_t s);
 size_t simt_backward_workspace(int total_tokens, int num_heads);
-cudaError_t launch_simt_backward(const BwdArgs& a, bool sparse, bool allow_mma, cudaStream_t s);
+// *path (may be null) receives the kernel family the dq and dk / dv passes use.
+cudaError_t launch_simt_backward(const BwdArgs& a, bool sparse, bool allow_mma, int* path,
+                                 cudaStream_t s);
 // The backward's tcgen05 passes: bf16, 64 heads, Dk <= 576 and Dv <= 512,
 // multiples of 64, 16-byte aligned operands; delta = the workspace's [T, H]
 // array.  dq query-major (tc_bwd_dq.cu); dk / dv key-major, a cluster of
@@ -119,6 +124,13 @@ cudaError_t launch_tc_full(const FullArgs& f, long long wait_limit, cudaStream_t
 
 // Records msg as the calling thread's hs_last_error() and returns st.
 hs_status report_error(hs_status st, const char* msg);
+
+// hs_block_score's host-side argument checks (no device work); HS_OK or the
+// status hs_block_score would return for them, with hs_last_error() set.
+hs_status check_score_args(const void* q, int64_t qrs, int64_t qhs, const void* k, int64_t krs,
+                           const int32_t* cu, int num_docs, int total_tokens, int max_seqlen,
+                           int num_heads, int dk, hs_dtype dtype, float scale, int block_size,
+                           const float* lse, const float* block_score, int nb_stride);
 
 // One thread waits (bounded) on an mbarrier nothing arrives at.
 cudaError_t launch_selftest_wait(long long limit_ns, int* status, cudaStream_t s);

@@ -12,9 +12,12 @@
 // library is loaded holds it (kStaticScratchBytes) until the process exits.
 // Host code cannot use the array's name as a device address; the address is
 // looked up once per device with cudaGetSymbolAddress, on the first call made
-// while that device is current.  Nothing is allocated, freed or zeroed by a
-// call: the kernel writes every scratch value before reading it, so the
-// contents left by a previous call do not matter.  All calls share the one
+// while that device is current, and kept for the life of the process (so
+// the library must not be used across a cudaDeviceReset, after which the
+// module is reloaded and the kept address would be stale).  Nothing is
+// allocated, freed or zeroed by a call: the kernel writes every scratch
+// value before reading it, so the contents left by a previous call do not
+// matter.  All calls share the one
 // array, so calls that may run at the same time on the GPU (different
 // streams, or different host threads) race on it and must be serialised by
 // the caller.
@@ -73,7 +76,16 @@ hs_status hs_block_score_static(const void* q, int64_t q_row_stride, int64_t q_h
                                 float softmax_scale, int block_size, float* lse,
                                 float* block_score, int nb_stride, float* block_lse,
                                 hs_stream_t stream) {
-  // size check first, on the host, before any device work
+  // the arguments first (a negative max_seqlen must not reach the sizing),
+  // then the size check, all on the host before any device work
+  hs_status r = hs::check_score_args(q, q_row_stride, q_head_stride, k, k_row_stride, cu_seqlens,
+                                     num_docs, total_tokens, max_seqlen, num_heads, dk, dtype,
+                                     softmax_scale, block_size, lse, block_score, nb_stride);
+  if (r != HS_OK) return r;
+  if (total_tokens == 0) return HS_OK;
+  // The limit follows from the shape alone, so it is conservative for a call
+  // that pointer alignment or its document count sends to the CUDA-core
+  // kernel, which needs no scratch.
   const size_t need = hs_workspace_size(HS_OP_BLOCK_SCORE, total_tokens, num_docs, max_seqlen,
                                         num_heads, dk, 0, dtype, block_size);
   if (need > kStaticScratchBytes) {
@@ -85,7 +97,7 @@ hs_status hs_block_score_static(const void* q, int64_t q_row_stride, int64_t q_h
     return hs::report_error(HS_ERR_WORKSPACE, msg);
   }
   void* scratch = nullptr;
-  hs_status r = scratch_address(&scratch);
+  r = scratch_address(&scratch);
   if (r != HS_OK) return r;
   return hs_block_score(q, q_row_stride, q_head_stride, k, k_row_stride, cu_seqlens, num_docs,
                         total_tokens, max_seqlen, num_heads, dk, dtype, softmax_scale,

@@ -449,7 +449,8 @@ size_t simt_backward_workspace(int total_tokens, int num_heads) {
   return (size_t)2 * total_tokens * num_heads * sizeof(float);
 }
 
-cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, bool allow_mma, cudaStream_t s) {
+cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, bool allow_mma, int* path,
+                                 cudaStream_t s) {
   BwdParams a{};
   a.p = b.p;
   a.idx = b.idx;
@@ -470,6 +471,7 @@ cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, bool allow_mma, 
     // tensor cores: dq and dk / dv on tcgen05 (else every pass on CUDA cores)
     const bool mma = allow_mma && tc_bwd_dq_supported(b.p) && tc_bwd_dkdv_supported(b.p) &&
                      (reinterpret_cast<uintptr_t>(b.dout) & 15) == 0;
+    if (path) *path = mma ? HS_PATH_MMA : HS_PATH_SIMT;
     cudaError_t e = sparse ? launch_typed<__nv_bfloat16, true>(a, !mma, s)
                            : launch_typed<__nv_bfloat16, false>(a, !mma, s);
     if (e != cudaSuccess || !mma) return e;
@@ -477,6 +479,7 @@ cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, bool allow_mma, 
     if (e != cudaSuccess) return e;
     return launch_tc_bwd_dkdv(b, sparse, a.delta, 0, s);
   }
+  if (path) *path = HS_PATH_SIMT;
   return sparse ? launch_typed<float, true>(a, true, s) : launch_typed<float, false>(a, true, s);
 }
 

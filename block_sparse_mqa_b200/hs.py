@@ -50,7 +50,7 @@ EXPORTS = (
     "hs_workspace_size", "hs_path", "hs_poll_status", "hs_set_force_simt",
     "hs_selftest_wait", "hs_status_string", "hs_last_error", "hs_version",
     "hs_block_score_static", "hs_sparse_mqa_bwd", "hs_swa_mqa_bwd",
-    "hs_block_score_attn_fwd", "hs_swa_layer_fwd",
+    "hs_block_score_attn_fwd", "hs_swa_layer_fwd", "hs_last_path",
 )
 
 
@@ -111,6 +111,8 @@ def lib() -> ctypes.CDLL:
     L.hs_status_string.restype = ctypes.c_char_p
     L.hs_last_error.argtypes = []
     L.hs_last_error.restype = ctypes.c_char_p
+    L.hs_last_path.argtypes = []
+    L.hs_last_path.restype = _int
     for fn in ("hs_block_score", "hs_select_topk", "hs_sparse_mqa_fwd", "hs_swa_mqa_fwd",
                "hs_poll_status", "hs_block_score_static", "hs_sparse_mqa_bwd",
                "hs_swa_mqa_bwd", "hs_block_score_attn_fwd", "hs_swa_layer_fwd"):
@@ -174,6 +176,13 @@ def selftest_wait(limit_ns: int, device=None):
 def path(op: int, dtype: torch.dtype, num_heads: int, dk: int, dv: int, block_size: int) -> int:
     code = HS_BF16 if dtype == torch.bfloat16 else HS_F32
     return lib().hs_path(op, code, num_heads, dk, dv, block_size)
+
+
+def last_path() -> int:
+    """Kernel family the calling thread's most recent successful call ran
+    (HS_PATH_*), -1 before the first one: tells a call that left the
+    tensor-core path because of its pointers or strides."""
+    return int(lib().hs_last_path())
 
 
 def poll_status(device=None):

@@ -135,6 +135,10 @@ typedef enum hs_kernel_path {
  *                hs_workspace_size(HS_OP_BLOCK_SCORE, ...) bytes (may be
  *                NULL when that size is 0).  Its contents on entry do not
  *                matter; concurrent calls must not share one workspace.
+ *                On the tensor-core path it is two [NBmax, 128] fp32 rows
+ *                per CTA, one CTA per SM: 128 is the row count of a query
+ *                tile (tokens x heads), independent of H (9.7 MB for
+ *                NBmax 64 on 148 SMs).
  *   block_size   16, 32, 64 or 128.
  */
 hs_status hs_block_score(const void* q, int64_t q_row_stride, int64_t q_head_stride,
@@ -161,6 +165,11 @@ hs_status hs_block_score(const void* q, int64_t q_row_stride, int64_t q_head_str
  *                ascending order, unused slots = -1.
  *   topk         1..256.  topk = 1 selects only the own block (the first
  *                block is then not forced).
+ *   NBmax = ceil(max_seqlen / block_size) <= 57344 (a row's keys are staged
+ *   in shared memory; e.g. documents up to 917504 tokens at block size 16);
+ *   longer rows are HS_ERR_UNSUPPORTED.
+ * One warp per query reads its row once; the selection is exact (no
+ * approximation) and bit-for-bit deterministic.
  */
 hs_status hs_select_topk(const float* block_score, int nb_stride,
                          const int32_t* cu_seqlens, int num_docs, int total_tokens,
@@ -317,7 +326,8 @@ hs_status hs_swa_mqa_bwd(const void* q, int64_t q_row_stride, int64_t q_head_str
  *   block_size   16, 32, 64 or 128.
  * bf16 with 64 heads, Dk and Dv multiples of 64 (Dk <= 576, Dv <= 512),
  * block sizes 32..128 and 16-byte aligned q, k, v, out run as ONE tcgen05
- * kernel (its scratch: two [NBmax, H] fp32 rows per SM).  Other inputs run
+ * kernel (its scratch: two [NBmax, 64] fp32 rows per SM, one per head of
+ * the 64).  Other inputs run
  * the attention and hs_block_score's kernel one after the other on the same
  * stream (same results, two passes over the logits).
  */
@@ -385,14 +395,21 @@ hs_status hs_swa_layer_fwd(const void* q, int64_t q_row_stride, int64_t q_head_s
  * library is loaded holds that array until the process exits).  It calls no
  * allocation or free routine.
  *
- *   - Problems whose scratch would exceed 16 MiB (hs_workspace_size of
- *     HS_OP_BLOCK_SCORE > 16 MiB; with 148 SMs that is about 110 key blocks
- *     per document, e.g. max_seqlen 7040 at block size 64) are rejected on
- *     the host with HS_ERR_WORKSPACE before any device work; use
- *     hs_block_score with a workspace for them.
+ *   - Arguments are validated first (the same checks as hs_block_score).
+ *     Then problems whose tensor-core scratch would exceed 16 MiB
+ *     (hs_workspace_size of HS_OP_BLOCK_SCORE > 16 MiB: two [NBmax, 128]
+ *     fp32 rows per SM, so with 148 SMs about 110 key blocks per document,
+ *     e.g. max_seqlen 7040 at block size 64) are rejected on the host with
+ *     HS_ERR_WORKSPACE before any device work; use hs_block_score with a
+ *     workspace for them.  The limit is applied from the shape alone, so it
+ *     is conservative for a call that would run the CUDA-core kernel (which
+ *     needs no scratch) because of its pointer alignment or document count.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) while that device is current; make that first
- *     call before any stream capture.
+ *     (cudaGetSymbolAddress) while that device is current and keeps it for
+ *     the life of the process; make that first call before any stream
+ *     capture, and do not use the library across a cudaDeviceReset (the
+ *     kept address would then be stale; the device status word of every
+ *     call is kept the same way).
  *   - All calls share the one array and nothing is cleared between calls
  *     (no scratch value is read before the kernel writes it, so the previous
  *     contents do not matter).  Calls that may overlap on the GPU (other
@@ -415,8 +432,21 @@ size_t hs_workspace_size(int op, int total_tokens, int num_docs, int max_seqlen,
                          int num_heads, int dk, int dv, hs_dtype dtype, int block_size);
 
 /* Which kernel family op would run for these parameters (hs_kernel_path),
- * or -1 when the parameters are unsupported. */
+ * or -1 when the parameters are unsupported.  It sees only the shape: a
+ * call whose pointers are not 16-byte aligned, whose strides are not
+ * multiples of 8 elements or (block scoring) whose cu_seqlens holds more
+ * than 1024 documents runs on the CUDA-core kernels even where hs_path
+ * says HS_PATH_TCGEN05; hs_last_path() reports what a call actually ran. */
 int hs_path(int op, hs_dtype dtype, int num_heads, int dk, int dv, int block_size);
+
+/* Kernel family (hs_kernel_path) that the calling thread's most recent
+ * successful compute call launched, or -1 before its first one.  A call
+ * that launches several kernels reports HS_PATH_SIMT when any part of its
+ * attention or scoring work ran on CUDA cores (top-k selection is always
+ * HS_PATH_SIMT: it is no contraction).  This is how a caller detects that a
+ * call left the tensor-core path because of its pointers or strides, which
+ * hs_path() cannot see.  Thread-local; failed calls leave it unchanged. */
+int hs_last_path(void);
 
 /* Synchronises `stream`, then returns and clears the device-side status
  * word (HS_OK when no kernel recorded a problem).  This is the only call

@@ -209,3 +209,45 @@ def test_swa_layer_rejects_bad_arguments():
     assert call(head=[p, 64 * 576, 576, p, 576, p, 500]) == hs.HS_ERR_INVALID_ARG
     assert call(outs=(p, None, p)) == hs.HS_ERR_INVALID_ARG
     assert call(outs=(p, p, None)) == hs.HS_ERR_INVALID_ARG
+
+
+def test_package_version_matches_library():
+    import block_sparse_mqa_b200 as pkg
+    v = hs.lib().hs_version()
+    assert pkg.__version__.split()[0] == "%d.%d.%d" % (v // 10000, v // 100 % 100, v % 100)
+
+
+def test_last_path_is_minus_one_before_any_compute_call():
+    # a rejected call does not change it; no call in this CPU process launches
+    assert _score(B=48) == hs.HS_ERR_UNSUPPORTED
+    assert hs.last_path() == -1
+
+
+def _static(**kw):
+    a = dict(q=1, qrs=64 * 576, qhs=576, k=1, krs=576, cu=1, nd=1, T=128, maxlen=128, H=64,
+             dk=576, dt=hs.HS_BF16, scale=0.0, B=64, lse=1, bs=1, nbs=2, blse=NULL)
+    a.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return hs.lib().hs_block_score_static(v(a["q"]), a["qrs"], a["qhs"], v(a["k"]), a["krs"],
+                                          v(a["cu"]), a["nd"], a["T"], a["maxlen"], a["H"],
+                                          a["dk"], a["dt"], a["scale"], a["B"], v(a["lse"]),
+                                          v(a["bs"]), a["nbs"], v(a["blse"]), None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(maxlen=-5), hs.HS_ERR_INVALID_ARG),   # must not wrap into a huge scratch size
+    (dict(maxlen=0), hs.HS_ERR_INVALID_ARG),
+    (dict(B=48), hs.HS_ERR_UNSUPPORTED),
+    (dict(q=None), hs.HS_ERR_INVALID_ARG),
+    (dict(nbs=1), hs.HS_ERR_INVALID_ARG),
+    (dict(T=100000, maxlen=100000, nbs=1563), hs.HS_ERR_WORKSPACE),
+])
+def test_static_block_score_validates_before_sizing(kw, code):
+    # arguments are checked on the host before the scratch size and before
+    # any CUDA call, so none of these touches a device
+    assert _static(**kw) == code
+    assert hs.lib().hs_last_error()
+
+
+def test_static_block_score_empty_input_is_a_no_op():
+    assert _static(T=0, nd=0, maxlen=0) == hs.HS_OK

@@ -54,13 +54,17 @@ def run_and_check(inp, B, K, W, rows=None, sink=True, scale=0.0, v=None, check_p
     rr = np.arange(T) if rows is None else np.asarray(rows)
     sc = None if scale == 0.0 else scale
 
+    ran = {}  # kernel family each call actually launched (hs_last_path)
     lse1, bs, blse = hs.hs_block_score(inp.q, inp.k, inp.cu_seqlens, inp.max_seqlen, B, scale,
                                        want_block_lse=rows is None)
+    ran["score"] = hs.last_path()
     idx = hs.hs_select_topk(bs, inp.cu_seqlens, inp.max_seqlen, B, K)
     out, lse = hs.hs_sparse_mqa_fwd(inp.q, inp.k, v_dev, idx, inp.cu_seqlens, inp.max_seqlen, B,
                                     sink_dev, scale)
+    ran["sparse"] = hs.last_path()
     wout, wlse = hs.hs_swa_mqa_fwd(inp.q, inp.k, v_dev, inp.cu_seqlens, inp.max_seqlen, W,
                                    sink_dev, scale)
+    ran["swa"] = hs.last_path()
     torch.cuda.synchronize()
     hs.poll_status()
 
@@ -102,7 +106,7 @@ def run_and_check(inp, B, K, W, rows=None, sink=True, scale=0.0, v=None, check_p
     P.check_out(wout[rows_t], ref4["out"], "swa out")
     P.check_lse(wlse[rows_t], ref4["lse"], "swa lse")
     return {"idx": idx, "out": out, "lse": lse, "swa_out": wout, "swa_lse": wlse, "bs": bs,
-            "lse1": lse1}
+            "lse1": lse1, "ran": ran}
 
 
 # ---------------------------------------------------------------------------
@@ -160,7 +164,9 @@ def test_v_aliases_latent_part_of_k():
     inp = _gpu_inputs(sum(docs), 64, 576, 512, torch.bfloat16, docs, seed=4)
     v_alias = inp.k[:, :512]  # absorbed-MLA: value = latent region of the key row
     assert v_alias.data_ptr() == inp.k.data_ptr()
-    run_and_check(inp, 64, 3, 128, v=v_alias)
+    res = run_and_check(inp, 64, 3, 128, v=v_alias)
+    assert res["ran"] == {"score": hs.HS_PATH_TCGEN05, "sparse": hs.HS_PATH_TCGEN05,
+                          "swa": hs.HS_PATH_TCGEN05}
 
 
 def test_strided_q_and_explicit_scale():
@@ -171,7 +177,28 @@ def test_strided_q_and_explicit_scale():
     big[:, :64, :576] = base.q
     base.q = big[:, :64, :576]
     assert base.q.stride() == (66 * 640, 640, 1)
-    run_and_check(base, 64, 3, 70, scale=0.03)
+    res = run_and_check(base, 64, 3, 70, scale=0.03)
+    assert set(res["ran"].values()) == {hs.HS_PATH_TCGEN05}
+
+
+def test_last_path_reports_a_stride_fallback():
+    """A q head stride that is not a multiple of 8 elements cannot be a TMA
+    operand, so those calls run on the CUDA-core kernels although hs_path
+    (which sees only the shape) names the tensor-core path; hs_last_path
+    reports what ran, and the results still match the oracle."""
+    docs = [150, 90]
+    T = sum(docs)
+    base = _gpu_inputs(T, 64, 576, 512, torch.bfloat16, docs, seed=5)
+    big = torch.zeros((T, 64, 580), device=DEV, dtype=torch.bfloat16)
+    big[:, :, :576] = base.q
+    base.q = big[:, :, :576]
+    assert base.q.stride(1) % 8 != 0
+    assert _expect_path(hs.HS_OP_SPARSE_MQA, base, 64) == hs.HS_PATH_TCGEN05
+    res = run_and_check(base, 64, 3, 70)
+    assert res["ran"] == {"score": hs.HS_PATH_SIMT, "sparse": hs.HS_PATH_SIMT,
+                          "swa": hs.HS_PATH_SIMT}
+    hs.hs_select_topk(res["bs"], base.cu_seqlens, base.max_seqlen, 64, 3)
+    assert hs.last_path() == hs.HS_PATH_SIMT  # selection is never a contraction
 
 
 def test_other_head_counts_and_dims():
