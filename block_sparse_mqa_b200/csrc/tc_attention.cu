@@ -115,6 +115,7 @@ struct Shared {
   uint64_t qfull[kMaxQChunks], qempty[kMaxQChunks];
   uint64_t sfull[2], sempty[2];
   uint64_t pfull, pvdone, ofull, oempty, drain, drain_pv;
+  uint64_t ochunk[4];        // O^T chunk c read out of TMEM (early epilogue)
   uint64_t rv[2];            // rendezvous inside softmax warpgroup wg (128 threads)
   uint64_t rv_all;           // rendezvous of both softmax warpgroups (full-layer mode)
   float red[2][4][32];       // [warpgroup][warp][lane] partial reductions
@@ -184,6 +185,53 @@ __device__ __forceinline__ TokenPlan plan_token(const AttnParams& p, int t, bool
       else if (b >= 0) bad = true;
     }
     if (bad && report) record_status(p.status, HS_ERR_INVALID_INDEX);
+    tp.nsel = n;
+    const int per = kTile / p.B;
+    tp.ntile = (n + per - 1) / per;
+  } else {
+    tp.wlo = max(tp.bos, t - p.window + 1);
+    tp.nkeys = t - tp.wlo + 1;
+    tp.ntile = (tp.nkeys + kTile - 1) / kTile;
+  }
+  return tp;
+}
+
+// The same plan computed by a whole warp (every lane calls it and gets the
+// result): the idx row is read with one coalesced load per 32 entries and
+// the index rule is evaluated per lane, the raw entry before it coming from
+// the neighbouring lane.  When `list` is not null the selected blocks are
+// written to it in order (compacted by ballot).  One L2 round trip per 32
+// entries instead of a serial walk over the row.
+template <bool kSparse>
+__device__ __forceinline__ TokenPlan plan_token_warp(const AttnParams& p, int t, bool report,
+                                                     int* list) {
+  const int lane = threadIdx.x & 31;
+  TokenPlan tp;
+  tp.ok = find_doc(p.cu, p.num_docs, p.T, p.max_seqlen, t, tp.bos, tp.eos,
+                   (report && lane == 0) ? p.status : nullptr);
+  tp.bq = tp.ok ? (t - tp.bos) / p.B : 0;
+  tp.wlo = 0;
+  tp.nkeys = 0;
+  tp.nsel = 0;
+  tp.ntile = 0;
+  if (!tp.ok) return tp;
+  if (kSparse) {
+    const int32_t* row = p.idx + (int64_t)t * p.topk;
+    int n = 0, prev_last = 0;
+    bool bad = false;
+    for (int base = 0; base < p.topk; base += 32) {
+      const int s = base + lane;
+      const int b = s < p.topk ? __ldg(row + s) : -1;
+      int prev = __shfl_up_sync(0xffffffffu, b, 1);
+      if (lane == 0) prev = prev_last;  // the previous 32 entries' last one
+      const bool v = b >= 0 && b <= tp.bq && (s == 0 || b > prev);
+      const unsigned m = __ballot_sync(0xffffffffu, v);
+      if (list && v) list[n + __popc(m & ((1u << lane) - 1u))] = b;
+      n += __popc(m);
+      bad = __any_sync(0xffffffffu, b >= 0 && !v) || bad;
+      prev_last = __shfl_sync(0xffffffffu, b, 31);
+    }
+    if (bad && report && lane == 0) record_status(p.status, HS_ERR_INVALID_INDEX);
     tp.nsel = n;
     const int per = kTile / p.B;
     tp.ntile = (n + per - 1) / per;
@@ -265,6 +313,10 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
   constexpr bool kSparse = kMode == kModeSparse;
   constexpr bool kFull = kMode == kModeFull;
   constexpr bool kCombine = kMode == kModeSwaLayer;
+  // The plain modes defer a token's epilogue until the next token's first P
+  // tile is written, and release O^T chunk by chunk to that token's first PV
+  // (the other modes stage their output through the P^T buffer).
+  constexpr bool kEarly = kMode == kModeSwa || kMode == kModeSparse;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -296,6 +348,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
     mbar_init(&sh->pvdone, 1);
     mbar_init(&sh->ofull, 1);
     mbar_init(&sh->oempty, 256);
+    for (int c = 0; c < 4; ++c) mbar_init(&sh->ochunk[c], 256);
     mbar_init(&sh->drain, 1);
     mbar_init(&sh->drain_pv, 1);
     fence_barrier_init();
@@ -369,19 +422,10 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
     };
     const int nst = is_v ? p.nvc : (p.nck + 1) / 2;  // stages per tile
     for (int t = blockIdx.x; t < p.T && !stop; t += G) {
-      const TokenPlan tp = plan_token<kSparse>(p, t, lane == 0 && !is_v);
+      // the token's plan and selected blocks (plist), read by the whole warp
+      const TokenPlan tp = plan_token_warp<kSparse>(p, t, !is_v, kSparse ? plist : nullptr);
       if (!tp.ok || tp.ntile == 0) continue;
-      if (kSparse) {  // this token's selected blocks, once
-        if (lane == 0) {
-          const int32_t* row = p.idx + (int64_t)t * p.topk;
-          int n = 0;
-          for (int s2 = 0; s2 < p.topk; ++s2) {
-            int b;
-            if (entry_ok(row, s2, tp.bq, b)) plist[n++] = b;
-          }
-        }
-        __syncwarp();
-      }
+      __syncwarp();  // plist complete before any lane reads it
       if (!is_v) {
         // Q_t chunks (lane c loads chunk c), each as soon as the previous
         // token's last QK released it
@@ -474,6 +518,10 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         tc_fence_after();
         for (int c = 0; c < p.nvc; ++c) {
           if (!mbar_wait_spin(&sh->vfull[slot], ph, lim)) return false;  // TMA stage
+          if (kEarly && first_tile && ntok > 0) {  // previous token's chunk c read out
+            if (!mbar_wait_spin(&sh->ochunk[c], (ntok - 1) & 1, lim)) return false;
+            tc_fence_after();
+          }
           const uint64_t a0 = ring_desc_v + (uint64_t)((slot * kSlotBytes) >> 4);
           const uint32_t d = tmem + c * kH;
           if (first_tile) pv_run<true>(d, a0, p_desc, id_pv);
@@ -486,6 +534,8 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         issued = true;
         return true;
       };
+      // lane 0 alone walks the tokens (the other lanes of the warp stay idle:
+      // divergent work beside the issuing lane was measured to slow MMA issue)
       for (int t = blockIdx.x; t < p.T && !stop; t += G) {
         const TokenPlan tp = plan_token<kSparse>(p, t, false);
         if (!tp.ok || tp.ntile == 0) continue;
@@ -495,12 +545,16 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           ++qtok;
         } else {
           // O^T of the previous token must have been read out before PV(0)
-          if (ntok > 0 && !mbar_wait(&sh->oempty, (ntok - 1) & 1, lim)) { stop = true; break; }
+          // (the plain modes wait per chunk inside pv)
+          if (!kEarly && ntok > 0 && !mbar_wait(&sh->oempty, (ntok - 1) & 1, lim)) {
+            stop = true;
+            break;
+          }
           tc_fence_after();
           for (int i = 0; i < tp.ntile; ++i)
             if (!pv(i == 0)) { stop = true; break; }
           if (stop) break;
-          umma_commit(&sh->ofull);
+          if (!kEarly) umma_commit(&sh->ofull);
           ++ntok;
         }
       }
@@ -529,8 +583,39 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
     const int nbt = kFull ? kTile / p.B : 0;
     const int wpb = kFull ? p.B / 32 : 1;
     float m_used = 0.f;
+    // Plain modes: the token whose output is still in TMEM (-1: none).  Its
+    // epilogue runs once the next token's first P tile is written: each
+    // 128-row dv chunk of O^T is read into registers, released at once to the
+    // next token's first PV (ochunk[c]), normalised by the token's sh->lsum
+    // and stored as bf16 straight to out (a warp writes 32 consecutive dv of
+    // one head per store).  The last PV of that token must be complete.
+    int pend_t = -1;
+    auto early_epilogue = [&]() {
+      __nv_bfloat16* const obase = p.out + ((int64_t)pend_t * kH + hb) * dvs;
+      float ls[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) ls[k] = sh->lsum[hb + k];
+      for (int c = 0; c < p.nvc; ++c) {
+        uint32_t w[32];
+        tmem_ld32(lane_base + c * kH + hb, w);
+        tmem_ld_wait();
+        reg_fence(w);
+        tc_fence_before();
+        mbar_arrive(&sh->ochunk[c]);
+        const int col = c * 128 + r;
+        if (col < dvs) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            obase[(int64_t)k * dvs + col] = __float2bfloat16_rn(__uint_as_float(w[k]) * ls[k]);
+        }
+      }
+      pend_t = -1;
+    };
     for (int t = blockIdx.x; t < p.T && ok && !aborted(sh); t += G) {
-      const TokenPlan tp = plan_token<kSparse>(p, t, false);
+      // the token's plan; warp 0 of the group also compacts its selected
+      // blocks into blist
+      const TokenPlan tp =
+          plan_token_warp<kSparse>(p, t, false, (kSparse && g4 == 0) ? sh->blist[wg] : nullptr);
       if (!tp.ok) continue;
       float* const blkrow =
           kFull ? p.blk + ((size_t)blockIdx.x * 2 + (ntok & 1)) * (size_t)p.nbmax * kH : nullptr;
@@ -550,19 +635,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         if (r < 32) p.lse[(int64_t)t * kH + hb + r] = p.sink ? __ldg(p.sink + hb + r) : -INFINITY;
         continue;
       }
-      if (kSparse) {  // compact this token's selected blocks (warp 0 of the group)
-        if (g4 == 0) {
-          const int32_t* row = p.idx + (int64_t)t * p.topk;
-          int n = 0;
-          for (int base0 = 0; base0 < p.topk; base0 += 32) {
-            const int s2 = base0 + lane;
-            int b = -1;
-            const bool v = s2 < p.topk && entry_ok(row, s2, tp.bq, b);
-            const unsigned mask = __ballot_sync(0xffffffffu, v);
-            if (v) sh->blist[wg][n + __popc(mask & ((1u << lane) - 1u))] = b;
-            n += __popc(mask);
-          }
-        }
+      if (kSparse) {  // blist is complete for every warp of the group after this
         if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
       }
       if (kCombine) {  // this warpgroup's rows of prev towards L2 for the epilogue
@@ -651,11 +724,11 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         // on a token's first tile once BOTH warpgroups have finished staging
         // the previous token's output in the same buffer (each warpgroup's
         // staging half spans rows that hold the other warpgroup's P^T columns)
-        if (i > 0) {
+        if (i > 0 || (kEarly && pend_t >= 0)) {
           if (!mbar_wait(&sh->pvdone, npv & 1, lim)) { ok = false; break; }
           ++npv;
           tc_fence_after();
-        } else if (ntok > 0) {
+        } else if (!kEarly && ntok > 0) {
           if (!mbar_wait(&sh->oempty, (ntok - 1) & 1, lim)) { ok = false; break; }
         }
         if (resc) {  // rare: some head's running max rose; rescale its O^T columns
@@ -684,6 +757,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
         mbar_arrive(&sh->pfull);
+        if (kEarly && pend_t >= 0) early_epilogue();  // the previous token's output
       }
       if (!ok) break;
       // ---------------- epilogue: per-head sums, sink, normalisation
@@ -705,6 +779,14 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         }
         sh->lse2[hh] = M + fast_log2(den);
         p.lse[(int64_t)t * kH + hh] = sh->lse2[hh] * kLn2;
+      }
+      if (kEarly) {
+        ++ntok;
+        pend_t = t;
+        // lsum is visible to the whole warpgroup, and red / mrun / blist may
+        // be rewritten for the next token, only after this
+        if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
+        continue;
       }
       // the last PV of this token must be complete before O^T is read
       if (!mbar_wait(&sh->pvdone, npv & 1, lim)) { ok = false; break; }
@@ -818,6 +900,15 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       ++ntok;
       // lsum / mrun / blist are rewritten for the next token only after this
       if (!rendezvous(sh, wg, rvph, lim)) { ok = false; break; }
+    }
+    if (kEarly && ok && pend_t >= 0 && !aborted(sh)) {  // the last token's output
+      if (mbar_wait(&sh->pvdone, npv & 1, lim)) {
+        ++npv;
+        tc_fence_after();
+        early_epilogue();
+      } else {
+        ok = false;
+      }
     }
     if (!ok) give_up(sh, p.status);
     if (!kCombine && r == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");

