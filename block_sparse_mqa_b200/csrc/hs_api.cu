@@ -114,6 +114,19 @@ hs_status check_problem(hs::Problem& p, const void* q, int64_t qrs, int64_t qhs,
   return HS_OK;
 }
 
+// The backward's workspace: the delta / sink terms of every path, then (for
+// shapes the tensor-core passes take) the dk / dv pass's partial sums at a
+// 256-byte boundary.
+size_t bwd_simt_bytes(int total_tokens, int num_heads) {
+  return (hs::simt_backward_workspace(total_tokens, num_heads) + 255) & ~(size_t)255;
+}
+size_t bwd_workspace(int total_tokens, int num_heads, int dk, int dv, hs_dtype dtype) {
+  size_t need = bwd_simt_bytes(total_tokens, num_heads);
+  if (!g_force_simt.load() && hs::tc_backward_shape_ok(dtype, num_heads, dk, dv))
+    need += hs::tc_bwd_dkdv_workspace(total_tokens, dk, dv);
+  return need;
+}
+
 hs_status launched(cudaError_t e, const char* what) {
   if (e != cudaSuccess) return cuda_fail(e, what);
   return HS_OK;
@@ -212,10 +225,9 @@ int hs_path(int op, hs_dtype dtype, int num_heads, int dk, int dv, int block_siz
 
 size_t hs_workspace_size(int op, int total_tokens, int num_docs, int max_seqlen, int num_heads,
                          int dk, int dv, hs_dtype dtype, int block_size) {
-  (void)dv;
   if ((op == HS_OP_SPARSE_MQA_BWD || op == HS_OP_SWA_MQA_BWD) && total_tokens > 0 &&
       num_heads > 0)
-    return hs::simt_backward_workspace(total_tokens, num_heads);
+    return bwd_workspace(total_tokens, num_heads, dk, dv, dtype);
   if ((op != HS_OP_BLOCK_SCORE && op != HS_OP_BLOCK_SCORE_ATTN) || total_tokens <= 0 ||
       !valid_block(block_size))
     return 0;
@@ -548,13 +560,16 @@ static hs_status backward_common(hs::BwdArgs& a, bool sparse, const void* q, int
   a.dval = dval;
   a.dsink = dsink;
   if (total_tokens == 0) return HS_OK;
-  const size_t need = hs::simt_backward_workspace(total_tokens, num_heads);
+  const size_t need = bwd_workspace(total_tokens, num_heads, dk, dv, dtype);
   if (!workspace || workspace_bytes < need)
     return fail(HS_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
                 workspace ? workspace_bytes : (size_t)0);
   if ((reinterpret_cast<uintptr_t>(workspace) & 15) != 0)
     return fail(HS_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
   a.workspace = workspace;
+  a.dkdv_ws = need > bwd_simt_bytes(total_tokens, num_heads)
+                  ? static_cast<char*>(workspace) + bwd_simt_bytes(total_tokens, num_heads)
+                  : nullptr;
   r = status_ptr(&a.p.status);
   if (r != HS_OK) return r;
   int path = HS_PATH_SIMT;

@@ -77,6 +77,7 @@ struct BwdArgs {
   float* dval;
   float* dsink;        // may be null
   void* workspace;     // simt_backward_workspace() bytes
+  void* dkdv_ws;       // the tensor-core dk / dv pass's partial sums, or null
 };
 
 // Launchers; each returns cudaSuccess or the launch error.
@@ -99,6 +100,8 @@ cudaError_t launch_simt_backward(const BwdArgs& a, bool sparse, bool allow_mma, 
 bool tc_backward_shape_ok(hs_dtype dtype, int num_heads, int dk, int dv);
 bool tc_bwd_dq_supported(const Problem& p);
 bool tc_bwd_dkdv_supported(const Problem& p);
+// Bytes of the dk / dv pass's partial sums (per query range, per key row).
+size_t tc_bwd_dkdv_workspace(int total_tokens, int dk, int dv);
 cudaError_t launch_tc_bwd_dq(const BwdArgs& a, bool sparse, const float* delta,
                              long long wait_limit, cudaStream_t s);
 cudaError_t launch_tc_bwd_dkdv(const BwdArgs& a, bool sparse, const float* delta,

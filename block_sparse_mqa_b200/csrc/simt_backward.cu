@@ -470,7 +470,7 @@ cudaError_t launch_simt_backward(const BwdArgs& b, bool sparse, bool allow_mma, 
   if (b.p.dtype == HS_BF16) {
     // tensor cores: dq and dk / dv on tcgen05 (else every pass on CUDA cores)
     const bool mma = allow_mma && tc_bwd_dq_supported(b.p) && tc_bwd_dkdv_supported(b.p) &&
-                     (reinterpret_cast<uintptr_t>(b.dout) & 15) == 0;
+                     (reinterpret_cast<uintptr_t>(b.dout) & 15) == 0 && b.dkdv_ws != nullptr;
     if (path) *path = mma ? HS_PATH_MMA : HS_PATH_SIMT;
     cudaError_t e = sparse ? launch_typed<__nv_bfloat16, true>(a, !mma, s)
                            : launch_typed<__nv_bfloat16, false>(a, !mma, s);

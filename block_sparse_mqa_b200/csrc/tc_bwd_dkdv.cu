@@ -32,6 +32,7 @@
 // are deterministic.
 // All waits are bounded (HS_ERR_TIMEOUT).
 
+#include <algorithm>
 #include <cooperative_groups.h>
 #include <math.h>
 
@@ -72,7 +73,39 @@ struct DkdvParams {
   float* dval;
   int* status;
   long long wait_ns;
+  // work items: (32-key tile, query range) pairs, range-major
+  int rlen, nrange;    // query-range length, number of ranges
+  int nitems;          // items that can hold members (see item_of)
+  float* part;         // [nrange][T][Dk + Dv] partial sums of the items (fp32)
 };
+
+// The tiles whose keys a query in [r0, r1) can attend: every earlier tile for
+// block-sparse attention, the tiles within one window before it for SWA.
+__host__ __device__ __forceinline__ void range_tiles(bool sparse, int rg, int rlen, int T,
+                                                     int window, int& tlo, int& thi) {
+  const int r0 = rg * rlen, r1 = min(T, r0 + rlen);
+  thi = (r1 + kKT - 1) / kKT;
+  tlo = sparse ? 0 : max(0, (r0 - window - kKT + 1) / kKT);
+  if (tlo > thi) tlo = thi;
+}
+
+// Work item k -> (tile, range): range-major, so the clusters that run at the
+// same time take members from the same range of queries (whose q_t and
+// dout_t then stay in L2), and a tile every query selects is spread over all
+// ranges instead of one cluster.
+__host__ __device__ __forceinline__ bool item_of(bool sparse, int k, int rlen, int nrange, int T,
+                                                 int window, int& tile, int& rg) {
+  for (rg = 0; rg < nrange; ++rg) {
+    int tlo, thi;
+    range_tiles(sparse, rg, rlen, T, window, tlo, thi);
+    if (k < thi - tlo) {
+      tile = tlo + k;
+      return true;
+    }
+    k -= thi - tlo;
+  }
+  return false;
+}
 
 struct Shared {
   uint64_t tile_full, sdp_full, sdp_empty, pds_full, pds_free, acc_done;
@@ -187,13 +220,23 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap kmap,
   // The tile, segment and candidate-chunk loops depend only on the inputs,
   // never on a CTA's own failures: every CTA of a cluster meets every cluster
   // barrier.  A CTA that gave up skips its members' work.
-  for (int tile = blockIdx.x / csize; tile * kKT < NT; tile += ncl) {
+  for (int item = blockIdx.x / csize; item < p.nitems; item += ncl) {
+    int tile, rg;
+    if (!item_of(kSparse, item, p.rlen, p.nrange, NT, p.window, tile, rg)) break;
+    const int r0 = rg * p.rlen, r1 = min(NT, r0 + p.rlen);  // this item's queries
     const int j1 = min(NT, tile * kKT + kKT);
     for (int s0 = tile * kKT; s0 < j1;) {  // one document segment at a time
       int bos, eos;
       // a malformed cu_seqlens fails alike in every CTA of the cluster
       if (!find_doc(p.cu, p.num_docs, NT, p.max_seqlen, s0, bos, eos, p.status)) break;
       const int s1 = min(j1, eos), n = s1 - s0;
+      // the segment's candidate queries [s0, tend) inside this item's range
+      const int tend_all = kSparse ? eos : min(eos, s1 - 1 + p.window);
+      const int c_lo = max(s0, r0), tend = min(tend_all, r1);
+      if (c_lo >= tend) {  // none: no partial sum for this segment and range
+        s0 = s1;
+        continue;
+      }
       // the segment's K and V rows (32 from s0; rows past the segment are
       // never a member's key; rows past T are zero-filled)
       if (warp == 0 && lane == 0) {
@@ -206,10 +249,9 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap kmap,
       ++ntile_loads;
       bool tile_waited = false;
       bool any = false;
-      const int tend = kSparse ? eos : min(eos, s1 - 1 + p.window);
       const int b_lo = kSparse ? (s0 - bos) / p.B : 0;
       const int b_hi = kSparse ? (s1 - 1 - bos) / p.B : 0;
-      for (int c0 = s0; c0 < tend; c0 += kThreads) {
+      for (int c0 = c_lo; c0 < tend; c0 += kThreads) {
         // candidate query t = c0 + tid: which of the segment's keys it attends
         const int t = c0 + tid;
         uint32_t mask = 0;
@@ -444,10 +486,7 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap kmap,
         const int kk = crank + (e / W) * csize, col = e - (e / W) * W;
         float sum = 0.f;
         for (int rr = 0; rr < csize; ++rr) sum += cl.map_shared_rank(part, rr)[kk * W + col];
-        if (col < dk)
-          p.dkey[(int64_t)(s0 + kk) * dk + col] = p.scale * sum;
-        else
-          p.dval[(int64_t)(s0 + kk) * dv + (col - dk)] = sum;
+        p.part[((int64_t)rg * NT + s0 + kk) * W + col] = sum;  // this range's share
       }
       cl.sync();  // no CTA reuses its shared memory while another still reads it
       s0 = s1;
@@ -464,7 +503,48 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap kmap,
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+// dk / dv from the items' partial sums: each key adds its rows over the
+// ranges its candidate queries fall in (the span the items used), in
+// increasing range order, and dk is scaled.
+template <bool kSparse>
+__global__ void __launch_bounds__(256) dkdv_reduce_kernel(const DkdvParams p) {
+  const int W = p.dk + p.dv;
+  const int64_t total = (int64_t)p.T * W;
+  for (int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * 256) {
+    const int j = (int)(e / W), col = (int)(e - (int64_t)j * W);
+    int bos, eos;
+    float sum = 0.f;
+    if (find_doc(p.cu, p.num_docs, p.T, p.max_seqlen, j, bos, eos, nullptr)) {
+      const int tile0 = (j / kKT) * kKT;
+      const int s0 = max(bos, tile0), s1 = min(tile0 + kKT, eos);
+      const int tend = kSparse ? eos : min(eos, s1 - 1 + p.window);
+      for (int rg = s0 / p.rlen; rg < p.nrange && rg * p.rlen < tend; ++rg)
+        sum += __ldcs(p.part + ((int64_t)rg * p.T + j) * W + col);
+    }
+    if (col < p.dk)
+      p.dkey[(int64_t)j * p.dk + col] = p.scale * sum;
+    else
+      p.dval[(int64_t)j * p.dv + (col - p.dk)] = sum;
+  }
+}
+
+// Query-range length and count of the work items: ranges of at least 512
+// queries (q_t and dout_t of one range, ~70 MB at 64 heads x 1088, fit in
+// L2), at most 8 of them (which bounds the partial-sum workspace).
+void range_split(int T, int& rlen, int& nrange) {
+  rlen = (T + 7) / 8;
+  if (rlen < 512) rlen = 512;
+  nrange = T > 0 ? (T + rlen - 1) / rlen : 0;
+}
+
 }  // namespace
+
+size_t tc_bwd_dkdv_workspace(int total_tokens, int dk, int dv) {
+  int rlen, nrange;
+  range_split(total_tokens, rlen, nrange);
+  return (size_t)nrange * (size_t)total_tokens * (size_t)(dk + dv) * sizeof(float);
+}
 
 bool tc_backward_shape_ok(hs_dtype dtype, int num_heads, int dk, int dv) {
   return dtype == HS_BF16 && num_heads == kH && dk % 64 == 0 && dk >= 64 && dk <= 64 * kMaxQC &&
@@ -529,11 +609,20 @@ cudaError_t launch_tc_bwd_dkdv(const BwdArgs& b, bool sparse, const float* delta
   a.dval = b.dval;
   a.status = p.status;
   a.wait_ns = wait_limit > 0 ? wait_limit : kDefaultWaitNs;
+  range_split(p.total_tokens, a.rlen, a.nrange);
+  a.nitems = 0;
+  for (int rg = 0; rg < a.nrange; ++rg) {
+    int tlo, thi;
+    range_tiles(sparse, rg, a.rlen, p.total_tokens, a.window, tlo, thi);
+    a.nitems += thi - tlo;
+  }
+  a.part = static_cast<float*>(b.dkdv_ws);
+  if (!a.part) return cudaErrorInvalidValue;
   auto kern = sparse ? tc_bwd_dkdv_kernel<true> : tc_bwd_dkdv_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int tiles = (p.total_tokens + kKT - 1) / kKT;
+  const int items = a.nitems;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -545,14 +634,24 @@ cudaError_t launch_tc_bwd_dkdv(const BwdArgs& b, bool sparse, const float* delta
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cfg.gridDim = dim3(tiles * kCluster);
+  cfg.gridDim = dim3(items * kCluster);
   int nclusters = 0;
   if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters < 1) {
     (void)cudaGetLastError();
-    attr[0].val.clusterDim.x = 1;  // single CTAs: each takes every member of its tile
-    cfg.gridDim = dim3(tiles);
+    attr[0].val.clusterDim.x = 1;  // single CTAs: each takes every member of its item
+    cfg.gridDim = dim3(items);
   }
-  return cudaLaunchKernelEx(&cfg, kern, kmap, vmap, qmap, dmap, a);
+  if (items > 0) {
+    cudaError_t le = cudaLaunchKernelEx(&cfg, kern, kmap, vmap, qmap, dmap, a);
+    if (le != cudaSuccess) return le;
+  }
+  const int64_t total = (int64_t)p.total_tokens * (p.dk + p.dv);
+  const int rgrid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sm_count() * 8);
+  if (sparse)
+    dkdv_reduce_kernel<true><<<rgrid, 256, 0, s>>>(a);
+  else
+    dkdv_reduce_kernel<false><<<rgrid, 256, 0, s>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace hs

@@ -253,17 +253,22 @@ hs_status hs_swa_mqa_fwd(const void* q, int64_t q_row_stride, int64_t q_head_str
  *                        dval into those columns of dkey)
  *   dsink      [H], or NULL to skip; ignored when sink is NULL.
  *   workspace  device scratch of at least hs_workspace_size(
- *              HS_OP_SPARSE_MQA_BWD, ...) bytes (8 * T * H), 16-byte
- *              aligned; its contents on entry do not matter; concurrent
- *              calls must not share one.  A missing or short workspace is
- *              HS_ERR_WORKSPACE before any device work.
+ *              HS_OP_SPARSE_MQA_BWD, ...) bytes, 16-byte aligned; its
+ *              contents on entry do not matter; concurrent calls must not
+ *              share one.  A missing or short workspace is HS_ERR_WORKSPACE
+ *              before any device work.  Size: 8 * T * H rounded up to 256,
+ *              plus, for shapes the tensor-core passes take, the dk / dv
+ *              pass's fp32 partial sums, nrange * T * (Dk + Dv) * 4 bytes,
+ *              with nrange = ceil(T / max(512, ceil(T / 8))) <= 8 query
+ *              ranges (143 MB at T = 4096, Dk 576, Dv 512).
  * idx entries follow the forward's rule; offending entries are skipped and
  * reported as HS_ERR_INVALID_INDEX.  Results are deterministic (every sum
  * runs in a fixed order).  bf16 inputs with 64 heads and Dk, Dv multiples of
  * 64 (Dk <= 576, Dv <= 512, 16-byte aligned) run on tcgen05 tensor cores
  * (hs_path: HS_PATH_MMA); other inputs on CUDA cores.  The dk / dv pass is a
- * four-CTA cluster kernel that falls back to single CTAs where the device
- * cannot place the cluster.
+ * four-CTA cluster kernel (single CTAs where the device cannot place the
+ * cluster) whose work items are (32-key tile, query range) pairs; their
+ * partial sums are added per key in a fixed range order by a second kernel.
  */
 hs_status hs_sparse_mqa_bwd(const void* q, int64_t q_row_stride, int64_t q_head_stride,
                             const void* k, int64_t k_row_stride,

@@ -116,8 +116,17 @@ def test_backward_rejects_bad_arguments():
     ws = ctypes.c_void_p(256)  # 16-byte aligned stand-in
     T, H = 100, 64
     need = L.hs_workspace_size(hs.HS_OP_SPARSE_MQA_BWD, T, 1, 100, H, 576, 512, hs.HS_BF16, 64)
-    assert need == 8 * T * H
+    # delta / sink terms (8 T H, to 256 bytes), then the dk / dv pass's fp32
+    # partial sums for its query ranges (ranges of >= 512 queries, <= 8)
+    rlen = max(512, -(-T // 8))
+    nrange = -(-T // rlen)
+    assert need == (8 * T * H + 255) // 256 * 256 + nrange * T * (576 + 512) * 4
     assert L.hs_workspace_size(hs.HS_OP_SWA_MQA_BWD, T, 1, 100, H, 576, 512, hs.HS_BF16, 64) == need
+    big = L.hs_workspace_size(hs.HS_OP_SPARSE_MQA_BWD, 65536, 1, 65536, H, 576, 512, hs.HS_BF16, 64)
+    assert big == 8 * 65536 * H + 8 * 65536 * (576 + 512) * 4  # 8 ranges of 8192
+    # CUDA-core shapes need only the delta / sink terms
+    assert L.hs_workspace_size(hs.HS_OP_SPARSE_MQA_BWD, T, 1, 100, H, 576, 512, hs.HS_F32, 64) \
+        == 8 * T * H
     assert L.hs_path(hs.HS_OP_SPARSE_MQA_BWD, hs.HS_BF16, H, 576, 512, 64) == hs.HS_PATH_MMA
     assert L.hs_path(hs.HS_OP_SWA_MQA_BWD, hs.HS_F32, H, 576, 512, 64) == hs.HS_PATH_SIMT
     assert L.hs_path(hs.HS_OP_SWA_MQA_BWD, hs.HS_BF16, 20, 80, 48, 64) == hs.HS_PATH_SIMT
