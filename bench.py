@@ -116,6 +116,17 @@ def window_pairs(docs, W):
     return tot
 
 
+def select_bytes(docs, B, topk):
+    """Algorithmic bytes of step 2: each query t reads its candidates'
+    scores, blocks 0 .. bq(t) of its row (4 bytes each), and writes topk
+    ids (4 bytes each)."""
+    tot = 0
+    for n in docs:
+        full, rem = divmod(n, B)  # blocks with all B queries, then a partial one
+        tot += B * full * (full + 1) // 2 + rem * (full + 1)
+    return 4.0 * tot + 4.0 * sum(docs) * topk
+
+
 def sparse_pairs(idx, cu, B):
     """sum_t |S_t| from the selected blocks (keys of each block up to t)."""
     idx = idx.cpu().numpy().astype(np.int64)
@@ -437,7 +448,7 @@ def run_ours(args, wl, world, rank):
         "swa": 2.0 * H * (wl.dk + wl.dv) * window_pairs(wl.docs(), wl.window),
     }
     nb = hs.nbmax(inp.max_seqlen, wl.block_size)
-    sel_bytes = 4.0 * sum(((n - 1) // wl.block_size + 1) * n for n in wl.docs()) + 4.0 * wl.total_tokens * wl.topk
+    sel_bytes = select_bytes(wl.docs(), wl.block_size, wl.topk)
     avg = {ph: statistics.mean(per_phase[p]) for p, ph in enumerate(Step.PHASES)}
     sustained = sum(avg.values()) >= LONG_STEP_MS and pk.get("bf16_tflops_sustained")
     tpk = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
@@ -593,8 +604,7 @@ def run_workloads(pk, flush, reps=3):
                 ms_tot = ms_score + ms_sel + ms_sp
                 peak, kind = frac_of(ms_tot)
                 pairs = sparse_pairs(st.idx, cu, wl.block_size)
-                sel_bytes = 4.0 * sum(((n - 1) // wl.block_size + 1) * n for n in wl.docs() if n) \
-                    + 4.0 * T * k
+                sel_bytes = select_bytes(wl.docs(), wl.block_size, k)
                 per_k[k] = {
                     "score": kern(ms_score, 2.0 * H * wl.dk * causal_pairs(wl.docs()), peak),
                     "select": {"ms": ms_sel, "gbs": sel_bytes / (ms_sel / 1e3) / 1e9,
