@@ -25,6 +25,15 @@
 // writes the chosen ids in ascending order.  With the early stop, theta may
 // sit below the m-th largest key, but only when exactly m keys reach it,
 // so no key equals the m-th without being taken: the set is the same.
+//
+// Rows of more than 64 candidates with m <= 32 first narrow the search:
+// each lane keeps its two largest keys, and the m-th largest p of those 64
+// values is found by the same search.  At least m distinct candidates reach
+// p, so the top m of the row, and every key equal to the m-th largest, are
+// among {key >= p}.  Those keys are copied, in block order, into a 64-entry
+// list in shared memory (two per lane), and the search and the output run
+// over that list instead of the whole row.  A row whose list would exceed
+// 64 entries (mass ties around p) takes the full search above.
 
 #include "hs_device.cuh"
 #include "hs_internal.h"
@@ -35,9 +44,13 @@ namespace {
 
 constexpr int kSelWarps = 8;         // queries per CTA
 constexpr int kRegChunks = 32;       // register path: up to 32 x 32 = 1024 candidates
+constexpr int kListSlots = 2;        // narrowed list: two keys per lane
+constexpr int kListCap = 32 * kListSlots;
 // Longer rows are staged in shared memory: at most kMaxSelectBlocks keys
-// (224 KB) for one warp, within the 227 KB a CTA may use.
-constexpr size_t kStageLimit = (size_t)kMaxSelectBlocks * sizeof(uint32_t);
+// (224 KB) plus the narrowed list (keys and ids) for one warp, within the
+// 227 KB a CTA may use.
+constexpr size_t kStageLimit = ((size_t)kMaxSelectBlocks + 2 * kListCap) * sizeof(uint32_t);
+static_assert(kStageLimit <= 232448, "staged row and list of one warp");
 
 // Monotone map of fp32 to uint32 (larger float -> larger integer).
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -135,6 +148,84 @@ __device__ __forceinline__ void write_selection(KeyAt key_at, int nch, int bq, b
   for (int i = pos + lane; i < topk; i += 32) out[i] = -1;  // only if pos < topk
 }
 
+// The narrowed selection for rows with 1 <= m <= 32 free slots (see the
+// file comment).  list_key / list_id: this warp's kListCap-entry buffers in
+// shared memory.  nch is a multiple of G (chunks past the row hold 0), so
+// the loops test their bound once per G chunks.  Returns false, having
+// written nothing, when more than kListCap keys reach the pivot; the caller
+// then runs the full search.
+template <int NCH, int G, typename KeyAt>
+__device__ __forceinline__ bool select_narrowed(KeyAt key_at, int nch, int m, int bq, bool two,
+                                                int32_t* out, uint32_t* list_key,
+                                                uint32_t* list_id) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t a = 0u, b = 0u;  // this lane's largest and second-largest key
+#pragma unroll
+  for (int i = 0; i < loop_bound<NCH>(); ++i) {
+    if (i % G == 0 && i >= nch) break;
+    const uint32_t k = key_at(i);
+    b = max(b, min(a, k));
+    a = max(a, k);
+  }
+  // pivot: the m-th largest of the 64 values, or 1 (every candidate) when
+  // fewer than m of them are candidates
+  uint32_t pivot = 1u;
+  const int nz = __popc(__ballot_sync(0xffffffffu, a != 0u)) +
+                 __popc(__ballot_sync(0xffffffffu, b != 0u));
+  if (nz >= m) {
+    int r_unused;
+    auto two_at = [&](int j) -> uint32_t { return j == 0 ? a : b; };
+    pivot = max(search_theta<kListSlots>(two_at, kListSlots, m, &r_unused), 1u);
+  }
+  // copy every key >= pivot into the list, in block order
+  int n = 0;
+#pragma unroll
+  for (int i = 0; i < loop_bound<NCH>(); ++i) {
+    if (i % G == 0 && i >= nch) break;
+    const uint32_t k = key_at(i);
+    const bool in = k >= pivot;
+    const unsigned mask = __ballot_sync(0xffffffffu, in);
+    const int o = n + __popc(mask & lt);
+    if (in && o < kListCap) {
+      list_key[o] = k;
+      list_id[o] = (uint32_t)(32 * i + lane);
+    }
+    n += __popc(mask);
+  }
+  if (n > kListCap) return false;
+  __syncwarp();
+  uint32_t lk[kListSlots], li[kListSlots];
+#pragma unroll
+  for (int j = 0; j < kListSlots; ++j) {
+    const int q = 32 * j + lane;
+    lk[j] = q < n ? list_key[q] : 0u;
+    li[j] = q < n ? list_id[q] : 0u;
+  }
+  int r;
+  auto list_at = [&](int j) -> uint32_t { return lk[j]; };
+  const uint32_t theta = search_theta<kListSlots>(list_at, kListSlots, m, &r);
+  // output: block 0 (forced), the chosen list entries in block order, bq
+  int pos = two ? 1 : 0, eq_seen = 0;
+#pragma unroll
+  for (int j = 0; j < kListSlots; ++j) {
+    const uint32_t key = lk[j];
+    const bool eq = key != 0u && key == theta;
+    const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = eq_seen + __popc(eq_mask & lt);
+    const bool sel = key != 0u && (key > theta || (eq && eq_rank < r));
+    const unsigned sel_mask = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[pos + __popc(sel_mask & lt)] = (int32_t)li[j];
+    pos += __popc(sel_mask);
+    eq_seen += __popc(eq_mask);
+  }
+  if (lane == 0) {  // pos == topk - 1: exactly m free blocks were taken
+    if (two) out[0] = 0;
+    out[pos] = bq;
+  }
+  return true;
+}
+
 // Per-query set-up shared by the kernels.  Returns false when the row is
 // finished already (no document, or every candidate fits).
 __device__ __forceinline__ bool begin_row(const int32_t* cu, int num_docs, int total_tokens,
@@ -156,7 +247,7 @@ __device__ __forceinline__ bool begin_row(const int32_t* cu, int num_docs, int t
 
 // Rows of up to 32 * NCH candidates: the keys live in registers.
 template <int NCH>
-__global__ void __launch_bounds__(kSelWarps * 32)
+__global__ void __launch_bounds__(kSelWarps * 32, NCH >= 32 ? 4 : 6)
 select_topk_reg_kernel(const float* __restrict__ block_score, int nb_stride,
                        const int32_t* __restrict__ cu, int num_docs, int total_tokens,
                        int max_seqlen, int block_size, int topk, int32_t* __restrict__ idx,
@@ -173,14 +264,24 @@ select_topk_reg_kernel(const float* __restrict__ block_score, int nb_stride,
   const int m = topk - (two ? 2 : 1);  // free slots
   const int nch = bq / 32 + 1;         // chunks holding candidates 0 .. bq
   const float* row = block_score + (int64_t)t * nb_stride;
+  // chunks are loaded in groups of four (NCH >= 4): entries past the row's
+  // last group are never read, those between nch and the group's end hold 0
+  constexpr int G = NCH >= 4 ? 4 : 1;
+  const int nchg = (nch + G - 1) / G * G;
   uint32_t key[NCH];
 #pragma unroll
   for (int i = 0; i < NCH; ++i) {  // one coalesced pass over the row
+    if (i % G == 0 && i >= nchg) break;
     const int c = 32 * i + lane;
-    key[i] = (i < nch && c >= flo && c < bq) ? order_key(__ldg(row + c)) : 0u;
+    key[i] = (c >= flo && c < bq) ? order_key(__ldg(row + c)) : 0u;
   }
   // every loop over the chunks is unrolled to NCH, so i is a constant here
   auto key_at = [&](int i) -> uint32_t { return key[i]; };
+  if (NCH > 2 && nch > 2 && m >= 1 && m <= 32) {
+    __shared__ uint32_t list[kSelWarps][2][kListCap];
+    const int w = threadIdx.x >> 5;
+    if (select_narrowed<NCH, G>(key_at, nchg, m, bq, two, out, list[w][0], list[w][1])) return;
+  }
   uint32_t theta = 0xffffffffu;  // no free slot (m = 0): no key is above theta
   int r = 0;
   if (m > 0) theta = search_theta<NCH>(key_at, nch, m, &r);
@@ -206,13 +307,16 @@ select_topk_long_kernel(const float* __restrict__ block_score, int nb_stride,
   const int m = topk - (two ? 2 : 1);
   const int nch = bq / 32 + 1;
   const float* row = block_score + (int64_t)t * nb_stride;
-  uint32_t* keys = stage + (size_t)w * slice;
+  uint32_t* keys = stage + (size_t)w * (slice + 2 * kListCap);
   for (int i = 0; i < nch; ++i) {  // one coalesced pass over the row
     const int c = 32 * i + lane;
     keys[c] = (c >= flo && c < bq) ? order_key(__ldg(row + c)) : 0u;
   }
   __syncwarp();
   auto key_at = [&](int i) -> uint32_t { return keys[32 * i + lane]; };
+  if (m >= 1 && m <= 32 &&
+      select_narrowed<0, 1>(key_at, nch, m, bq, two, out, keys + slice, keys + slice + kListCap))
+    return;
   uint32_t theta = 0xffffffffu;  // no free slot (m = 0): no key is above theta
   int r = 0;
   if (m > 0) theta = search_theta<0>(key_at, nch, m, &r);
@@ -249,7 +353,7 @@ cudaError_t launch_select_topk(const float* block_score, int nb_stride, const in
   // longer rows: one warp's slice of shared memory holds a row's keys (the
   // host has refused rows past kMaxSelectBlocks)
   const int slice = nch * 32;
-  const size_t per_warp = (size_t)slice * sizeof(uint32_t);
+  const size_t per_warp = ((size_t)slice + 2 * kListCap) * sizeof(uint32_t);
   if (per_warp > kStageLimit) return cudaErrorInvalidValue;
   int warps = (int)(kStageLimit / per_warp);
   if (warps > kSelWarps) warps = kSelWarps;

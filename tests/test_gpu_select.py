@@ -1,7 +1,11 @@
 """GPU parity of step 2 (hs_select_topk) on its own: score rows drawn here,
 not by step 1, so that rows of every length class meet the kernel (the
 register path for up to 32 x {1, 2, 4, 8, 16, 32} candidates and the
-shared-memory path past 1024), with many exact ties.
+shared-memory path past 1024), with many exact ties.  Rows of more than 64
+candidates with at most 32 free slots take the narrowed search (a pivot from
+each lane's two largest keys, then a 64-entry list); the "ties" rows
+overflow that list and take the full search, the "coarse" rows hold ties
+around the pivot that often still fit in it.
 
 Selection decides integers from fp32 scores, so both sides decide in fp32:
 the oracle sorts the float64 images of the same fp32 values, which order
@@ -29,6 +33,8 @@ def _scores(T, nb, kind, seed):
         return u.mul_(6.0).floor_()
     if kind == "flat":      # near-equal positive scores, as from N(0,1) inputs
         return u.mul_(2e-3).add_(1.0)
+    if kind == "coarse":    # 48 levels: ties at the k-th value, short lists
+        return u.mul_(48.0).floor_().add_(1.0)
     if kind == "mixed":     # exact zeros (underflow), tiny and large values
         z = torch.rand((T, nb), generator=g, device="cuda") < 0.2
         return u.mul_(105.0).sub_(100.0).exp_().masked_fill_(z, 0.0)
@@ -53,7 +59,7 @@ def _check(docs, B, K, kind, seed, rows=None):
     np.testing.assert_array_equal(idx[rt].cpu().numpy(), ref)
 
 
-@pytest.mark.parametrize("kind", ["ties", "flat", "mixed"])
+@pytest.mark.parametrize("kind", ["ties", "coarse", "flat", "mixed"])
 @pytest.mark.parametrize("B,K,docs", [
     (16, 4, [500, 0, 33]),          # up to 32 candidates: one register chunk
     (16, 2, [1000]),                 # k = 2: only the two forced blocks
@@ -63,6 +69,9 @@ def _check(docs, B, K, kind, seed, rows=None):
     (16, 37, [4096, 5]),             # 256: eight chunks
     (64, 100, [32768]),              # 512: sixteen chunks
     (16, 256, [16384]),              # 1024: thirty-two chunks, topk at its maximum
+    (64, 34, [65536]),               # 1024 candidates, m = 32: the narrowed search at its limit
+    (64, 35, [40000]),               # m = 33: the full search on the same chunk count
+    (32, 3, [20000, 3000]),          # m = 1
 ])
 def test_select_matches_oracle_register_path(kind, B, K, docs):
     T = sum(docs)
@@ -71,10 +80,11 @@ def test_select_matches_oracle_register_path(kind, B, K, docs):
     _check(docs, B, K, kind, seed=len(docs) * 1000 + K, rows=rows)
 
 
-@pytest.mark.parametrize("kind", ["ties", "flat", "mixed"])
+@pytest.mark.parametrize("kind", ["ties", "coarse", "flat", "mixed"])
 @pytest.mark.parametrize("B,K,docs,nrows", [
     (16, 32, [24000, 17], 800),      # 1500 candidates: shared-memory staging, 8 warps a CTA
     (16, 64, [320000], 120),         # 20000 candidates: 80 KB a row, 2 warps a CTA
+    (16, 30, [320000], 120),         # the same rows, m = 28: narrowed search from shared memory
 ])
 def test_select_matches_oracle_shared_memory_path(kind, B, K, docs, nrows):
     T = sum(docs)
