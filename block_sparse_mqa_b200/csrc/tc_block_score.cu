@@ -600,20 +600,22 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
       const int nbatch = (p.nbmax + 31) / 32;
       for (int bi = wg; bi < nbatch; bi += 2) {
         const int bb0 = bi * 32;
+        // all 32 workspace loads first: interleaved with the block_lse
+        // stores, which may alias them, they would run one L2 round trip at
+        // a time
         float v[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int b = bb0 + j;
-          float e = 0.f;
-          if (b <= bq) {
-            const float w = ws_row[(size_t)b * 128];
-            e = fast_exp2(w - lse2);
-            if (blo) blo[b] = w * kLn2;
-          } else if (blo && b < p.nbmax) {
-            blo[b] = -INFINITY;
+        for (int j = 0; j < 32; ++j) v[j] = bb0 + j <= bq ? ws_row[(size_t)(bb0 + j) * 128] : 0.f;
+        if (blo) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int b = bb0 + j;
+            if (b <= bq) blo[b] = v[j] * kLn2;
+            else if (b < p.nbmax) blo[b] = -INFINITY;
           }
-          v[j] = e;
         }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = bb0 + j <= bq ? fast_exp2(v[j] - lse2) : 0.f;
         const float s = transpose_reduce_sum(v);
         sh->red[wg][g4][lane] = s;
         mbar_arrive(&sh->epi_wg[wg]);
