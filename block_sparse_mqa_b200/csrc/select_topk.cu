@@ -247,7 +247,7 @@ __device__ __forceinline__ bool begin_row(const int32_t* cu, int num_docs, int t
 
 // Rows of up to 32 * NCH candidates: the keys live in registers.
 template <int NCH>
-__global__ void __launch_bounds__(kSelWarps * 32, NCH >= 32 ? 4 : 6)
+__global__ void __launch_bounds__(kSelWarps * 32, NCH >= 32 ? 5 : 6)
 select_topk_reg_kernel(const float* __restrict__ block_score, int nb_stride,
                        const int32_t* __restrict__ cu, int num_docs, int total_tokens,
                        int max_seqlen, int block_size, int topk, int32_t* __restrict__ idx,
