@@ -158,9 +158,9 @@ __device__ __forceinline__ float transpose_reduce_sum(float (&v)[32]) {
 // One ring stage = NC (three, fewer in the last stage when Dk is not a
 // multiple of 192) 64-column K chunks = 4 NC MMAs (M=128, N=128, K=16) into S
 // accumulator d.  FIRST: the stage opens the S tile (its first MMA
-// overwrites d).  SS_FIRST: its first chunk is the shared-memory q chunk
-// (descriptor qd), the others come from TMEM q chunks tpos, tpos+1, ...
-template <bool FIRST, bool SS_FIRST, int NC = kChunksPerStage>
+// overwrites d).  The stage's chunks come from TMEM q chunks tpos, tpos+1,
+// ...; SS_LAST: its last chunk is the shared-memory q chunk (descriptor qd).
+template <bool FIRST, bool SS_LAST, int NC = kChunksPerStage>
 __device__ __forceinline__ void issue_stage(uint32_t d, uint32_t tmem, int tpos, uint64_t qd,
                                             uint64_t b0, uint32_t idesc) {
 #pragma unroll
@@ -169,7 +169,7 @@ __device__ __forceinline__ void issue_stage(uint32_t d, uint32_t tmem, int tpos,
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const uint32_t acc = (FIRST && c == 0 && k == 0) ? 0u : 1u;
-      if (SS_FIRST && c == 0)
+      if (SS_LAST && c == NC - 1)
         umma_ss(d, qd + 2 * k, bc + 2 * k, idesc, acc);
       else
         umma_ts(d, tmem + (uint32_t)((tpos + c) * 32 + k * 8), bc + 2 * k, idesc, acc);
@@ -276,6 +276,22 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
               for (int ch = 0; ch < p.nck; ++ch) tma_prefetch_3d(&qmap, ch * 64, 0, t2.t0);
             }
           }
+          // the tile's q chunks that live in TMEM pass through ring 0 (three
+          // per stage; MMA issuer 0 copies them into TMEM with tcgen05.cp):
+          // they need only ring slots, which the previous tile's last ring-0
+          // stages free.  The shared-memory chunk comes after them: its
+          // buffer is free only once both issuers' MMAs of the previous tile
+          // are complete.
+          for (int q0 = 0; q0 < p.nq_tmem; q0 += kChunksPerStage) {
+            const int n = min(kChunksPerStage, p.nq_tmem - q0);
+            uint8_t* dst = open_stage(n * kChunkBytes);
+            if (!dst) { stop = true; break; }
+            const int sl = r * kSlots + (int)kst;
+            for (int j = 0; j < n; ++j)
+              tma_load_3d(dst + j * kChunkBytes, &qmap, &sh->kfull[sl], (q0 + j) * 64, 0, tl.t0);
+            close_stage();
+          }
+          if (stop) break;
           if (p.nq_smem > 0) {
             if (qfills > 0 && !mbar_wait(&sh->qhi_empty, (qfills - 1) & 1, lim)) {
               stop = true;
@@ -287,21 +303,9 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
                           tl.t0);
             ++qfills;
           }
-          // the tile's q chunks that live in TMEM pass through ring 0 (three
-          // per stage); MMA issuer 0 copies them into TMEM with tcgen05.cp
-          for (int q0 = 0; q0 < p.nq_tmem; q0 += kChunksPerStage) {
-            const int n = min(kChunksPerStage, p.nq_tmem - q0);
-            uint8_t* dst = open_stage(n * kChunkBytes);
-            if (!dst) { stop = true; break; }
-            const int sl = r * kSlots + (int)kst;
-            for (int j = 0; j < n; ++j)
-              tma_load_3d(dst + j * kChunkBytes, &qmap, &sh->kfull[sl], (q0 + j) * 64, 0, tl.t0);
-            close_stage();
-          }
-          if (stop) break;
         }
         // this ring's key tiles: stages of three K chunks in the MMA's order,
-        // the shared-memory (RoPE) chunks first, then the TMEM chunks 0, 1, ...
+        // the TMEM chunks 0, 1, ... first, then the shared-memory (RoPE) chunk
         const int spt = (p.nck + kChunksPerStage - 1) / kChunksPerStage;  // stages per key tile
         for (int kt = 0; kt < nkt && !stop; ++kt) {
           if (((sbase + kt) & 1) != r) continue;
@@ -311,8 +315,7 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
             if (!dst) { stop = true; break; }
             const int sl = r * kSlots + (int)kst;
             for (int j = 0; j < nst; ++j) {
-              const int pos = st * kChunksPerStage + j;
-              const int ch = pos < p.nq_smem ? p.nq_tmem + pos : pos - p.nq_smem;
+              const int ch = st * kChunksPerStage + j;  // K chunk = q chunk position
               tma_load_2d(dst + j * kChunkBytes, &kmap, &sh->kfull[sl], ch * 64,
                           tl.bos + kt * kKeyTile);
             }
@@ -361,8 +364,7 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
         if (r == 0) {
           // q enters TMEM by tcgen05.cp from the ring, once every MMA of the
           // previous tile (which read the old q) has completed
-          if ((qtile > 0 && !mbar_wait_spin(&sh->qdone, (qtile - 1) & 1, lim)) ||
-              (p.nq_smem > 0 && !mbar_wait(&sh->qhi_full, qtile & 1, lim))) {
+          if (qtile > 0 && !mbar_wait_spin(&sh->qdone, (qtile - 1) & 1, lim)) {
             ok = false;
             break;
           }
@@ -389,14 +391,16 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
         } else {
           // every tile's phases, even with no key tile of this parity: a
           // parity wait must never run two phases ahead of its barrier
-          if (!mbar_wait_spin(&sh->qready, qtile & 1, lim) ||
-              (p.nq_smem > 0 && !mbar_wait(&sh->qhi_full, qtile & 1, lim))) {
+          if (!mbar_wait_spin(&sh->qready, qtile & 1, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
         }
         const int spt = (p.nck + kChunksPerStage - 1) / kChunksPerStage;
+        // the shared-memory q chunk is waited for once per tile, before its
+        // first use (the last stage of a key tile), or at the tile's end
+        bool qhi_seen = p.nq_smem == 0;
         for (int kt = 0; kt < nkt && ok; ++kt) {
           if (((sbase + kt) & 1) != r) continue;
           if (!mbar_wait_spin(&sh->sempty[r], (myidx & 1) ^ 1, lim)) {
@@ -415,13 +419,21 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
             // 12 MMAs without a branch between them (a branch between two
             // tcgen05.mma costs about half the issue rate); one stage pattern
             // is chosen per stage
-            const int tpos = st * kChunksPerStage - p.nq_smem;  // first TMEM chunk
+            const int tpos = st * kChunksPerStage;  // first TMEM chunk
             // a shorter last stage (Dk not a multiple of 192) only occurs
-            // without a shared-memory q chunk (that needs 9 chunks)
+            // without a shared-memory q chunk (that needs 9 chunks: the last
+            // stage is then TMEM chunks 6, 7 and the shared-memory chunk)
             const int nst = min(kChunksPerStage, p.nck - st * kChunksPerStage);
-            if (st == 0 && p.nq_smem > 0)
-              issue_stage<true, true>(d, tmem, tpos, qhi_desc[0], b0, idesc);
-            else if (nst == kChunksPerStage) {
+            if (st == spt - 1 && p.nq_smem > 0) {
+              if (!qhi_seen) {
+                if (!mbar_wait(&sh->qhi_full, qtile & 1, lim)) {
+                  ok = false;
+                  break;
+                }
+                qhi_seen = true;
+              }
+              issue_stage<false, true>(d, tmem, tpos, qhi_desc[0], b0, idesc);
+            } else if (nst == kChunksPerStage) {
               if (st == 0) issue_stage<true, false>(d, tmem, tpos, 0, b0, idesc);
               else issue_stage<false, false>(d, tmem, tpos, 0, b0, idesc);
             } else if (nst == 2) {
@@ -440,6 +452,13 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
           ++myidx;
         }
         if (!ok) break;
+        // every tile's phase of the shared-memory chunk is waited for, even
+        // with no key tile of this parity (a parity wait must never run two
+        // phases ahead of its barrier)
+        if (!qhi_seen && !mbar_wait(&sh->qhi_full, qtile & 1, lim)) {
+          ok = false;
+          break;
+        }
         // this issuer is done with the tile's q (both commit; count 2)
         if (p.nq_smem > 0) umma_commit(&sh->qhi_empty);
         umma_commit(&sh->qdone);
