@@ -94,7 +94,7 @@ struct Shared {
   uint64_t kfull[kStages], kempty[kStages];
   uint64_t qhi_full, qhi_empty;  // the shared-memory q chunk (empty: both issuers)
   uint64_t qdone;                // a query tile's MMAs of both issuers have completed
-  uint64_t qready;               // issuer 0's copies of q into TMEM have completed
+  uint64_t qready;               // both issuers' copies of q into TMEM have completed
   uint64_t drain[2];
   uint64_t sfull[2], sempty[2];
   uint64_t epi_all;    // rendezvous of both softmax warpgroups (256 threads)
@@ -198,7 +198,7 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
     mbar_init(&sh->qhi_full, 1);
     mbar_init(&sh->qhi_empty, 2);
     mbar_init(&sh->qdone, 2);
-    mbar_init(&sh->qready, 1);
+    mbar_init(&sh->qready, 2);
     mbar_init(&sh->drain[0], 1);
     mbar_init(&sh->drain[1], 1);
     for (int b = 0; b < 2; ++b) {
@@ -241,7 +241,7 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
     const int r = warp == 0 ? 0 : 1;
     if (lane == 0) {
       tma_prefetch_desc(&kmap);
-      if (r == 0) tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&qmap);
       int fills[kSlots];
 #pragma unroll
       for (int s2 = 0; s2 < kSlots; ++s2) fills[s2] = 0;
@@ -276,14 +276,16 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
               for (int ch = 0; ch < p.nck; ++ch) tma_prefetch_3d(&qmap, ch * 64, 0, t2.t0);
             }
           }
-          // the tile's q chunks that live in TMEM pass through ring 0 (three
-          // per stage; MMA issuer 0 copies them into TMEM with tcgen05.cp):
-          // they need only ring slots, which the previous tile's last ring-0
-          // stages free.  The shared-memory chunk comes after them: its
-          // buffer is free only once both issuers' MMAs of the previous tile
-          // are complete.
-          for (int q0 = 0; q0 < p.nq_tmem; q0 += kChunksPerStage) {
-            const int n = min(kChunksPerStage, p.nq_tmem - q0);
+        }
+        {
+          // the tile's q chunks that live in TMEM: half of them pass through
+          // each ring (at most three per stage) and that ring's MMA issuer
+          // copies them into TMEM with tcgen05.cp.  They need only ring
+          // slots, which the previous tile's last stages of the ring free.
+          const int qlo = r == 0 ? 0 : (p.nq_tmem + 1) / 2;
+          const int qhi_end = r == 0 ? (p.nq_tmem + 1) / 2 : p.nq_tmem;
+          for (int q0 = qlo; q0 < qhi_end; q0 += kChunksPerStage) {
+            const int n = min(kChunksPerStage, qhi_end - q0);
             uint8_t* dst = open_stage(n * kChunkBytes);
             if (!dst) { stop = true; break; }
             const int sl = r * kSlots + (int)kst;
@@ -292,6 +294,10 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
             close_stage();
           }
           if (stop) break;
+        }
+        if (r == 0) {
+          // the shared-memory chunk comes after them: its buffer is free only
+          // once both issuers' MMAs of the previous tile are complete
           if (p.nq_smem > 0) {
             if (qfills > 0 && !mbar_wait(&sh->qhi_empty, (qfills - 1) & 1, lim)) {
               stop = true;
@@ -335,10 +341,11 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
     // ------------------------------------------------------------ MMA issuers
     // Issuer r issues the key tiles of global parity r from ring r into S
     // buffer r (the softmax warpgroup r reads it); two instruction streams,
-    // so each one's pipeline waits overlap the other's MMAs.  Issuer 0 also
-    // copies each query tile's q into TMEM, once both issuers' MMAs of the
-    // previous tile are complete (qdone counts both), and commits qready,
-    // which issuer 1 waits for before its first MMA of the tile.
+    // so each one's pipeline waits overlap the other's MMAs.  Each issuer
+    // also copies the half of a query tile's q that came through its ring
+    // into TMEM, once both issuers' MMAs of the previous tile are complete
+    // (qdone counts both), and commits qready; both wait for qready (count
+    // 2: both halves copied) before their first MMA of the tile.
     const int r = warp == 1 ? 0 : 1;
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
@@ -361,16 +368,18 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
         if (g >= total) continue;
         const Tile tl = tile_of(g, sh->prefix, nd, p.cu, p.tpt);
         const int nkt = (tl.tend - tl.bos + kKeyTile - 1) / kKeyTile;
-        if (r == 0) {
-          // q enters TMEM by tcgen05.cp from the ring, once every MMA of the
-          // previous tile (which read the old q) has completed
+        {
+          // this ring's half of q enters TMEM by tcgen05.cp, once every MMA
+          // of the previous tile (which read the old q) has completed
           if (qtile > 0 && !mbar_wait_spin(&sh->qdone, (qtile - 1) & 1, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          for (int q0 = 0; q0 < p.nq_tmem; q0 += kChunksPerStage) {
-            const int n = min(kChunksPerStage, p.nq_tmem - q0);
+          const int qlo = r == 0 ? 0 : (p.nq_tmem + 1) / 2;
+          const int qhi_end = r == 0 ? (p.nq_tmem + 1) / 2 : p.nq_tmem;
+          for (int q0 = qlo; q0 < qhi_end; q0 += kChunksPerStage) {
+            const int n = min(kChunksPerStage, qhi_end - q0);
             const int sl = r * kSlots + (int)kst;
             if (!mbar_wait_spin(&sh->kfull[sl], kph, lim)) {  // TMA stage
               ok = false;
@@ -386,11 +395,9 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
             next_slot();
           }
           if (!ok) break;
-          umma_commit(&sh->qready);  // arrives once the copies have completed
+          umma_commit(&sh->qready);  // arrives once this issuer's copies have completed
           issued = true;
-        } else {
-          // every tile's phases, even with no key tile of this parity: a
-          // parity wait must never run two phases ahead of its barrier
+          // both halves in TMEM (every tile's phase is waited for)
           if (!mbar_wait_spin(&sh->qready, qtile & 1, lim)) {
             ok = false;
             break;
