@@ -19,7 +19,8 @@
 //    each); three chunks form one 48 KB stage, so every pipeline wait of an
 //    MMA thread is followed by 12 M=128, N=128, K=16 MMAs issued without a
 //    branch between them (a branch between two MMAs costs about half the
-//    issue rate).  The shared-memory (RoPE) chunk goes first.  Key tiles
+//    issue rate).  The shared-memory (RoPE) chunk goes last, so that a query
+//    tile's first key tiles need not wait for it.  Key tiles
 //    alternate between two MMA-issuing threads, each with its own producer
 //    and two-slot ring and its own S buffer in TMEM: a wait costs one issuing
 //    thread a few hundred cycles (measured: the stage waits took ~650 of the
@@ -32,9 +33,11 @@
 //    L2 resident; halves alternate by query tile).  At the end of the tile each row has its LSE; the head
 //    sum of exp2(blockLSE - LSE) is a 32-lane transpose-reduction per warp
 //    plus a fixed-order sum over the warps of a token (deterministic).
-//  * Warps 0 / 10 = TMA producers of rings 0 / 1 (warp 0 also loads q),
-//    warps 1 / 11 = MMA issuers of key tiles of even / odd index (warp 1 also
-//    copies q into TMEM and owns TMEM), warps 2-9 = two softmax warpgroups
+//  * Warps 0 / 10 = TMA producers of rings 0 / 1 (each also loads half of
+//    the query tile's TMEM q chunks into its ring; warp 0 loads the RoPE
+//    chunk), warps 1 / 11 = MMA issuers of key tiles of even / odd index
+//    (each copies its ring's half of q into TMEM; warp 1 owns TMEM),
+//    warps 2-9 = two softmax warpgroups
 //    that take the alternate S tiles (one S buffer each) and share the
 //    epilogue.  Per-row running
 //    (max, sum) pairs of the two warpgroups are merged at the end of the
@@ -235,9 +238,9 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
   if (warp == 0 || warp == kProdB) {
     // ------------------------------------------------------------ producers
     // Producer r fills ring r with the stages of the key tiles whose global
-    // index (key tiles counted over this CTA's query tiles) has parity r;
-    // producer 0 also loads each query tile's q: the shared-memory chunk and,
-    // through ring 0, the chunks that go to TMEM.
+    // index (key tiles counted over this CTA's query tiles) has parity r,
+    // preceded in each query tile by its half of the tile's TMEM q chunks;
+    // producer 0 also loads the shared-memory (RoPE) q chunk.
     const int r = warp == 0 ? 0 : 1;
     if (lane == 0) {
       tma_prefetch_desc(&kmap);
