@@ -527,6 +527,44 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         return true;
       };
       // O^T += V_tile^T . P^T (waits for P of this tile); 8 MMAs per stage
+      // A token's middle tiles (neither its first nor its last) run the same
+      // stages without the first / last tile's q waits and releases, so that
+      // no branch on them sits between two stages' runs of MMAs.
+      auto qk_mid = [&]() -> bool {
+        const uint32_t buf = sidx & 1, use = sidx >> 1;
+        if (!mbar_wait_spin(&sh->sempty[buf], (use & 1) ^ 1, lim)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + kSCol + buf * kH;
+        for (int s = 0; s < (p.nck + 1) / 2; ++s) {
+          const int c0 = 2 * s;
+          const bool two = c0 + 1 < p.nck;
+          if (!mbar_wait_spin(&sh->kfull[slot], ph, lim)) return false;  // TMA stage
+          const uint64_t a = ring_desc_k + (uint64_t)((slot * kSlotBytes) >> 4);
+          const uint64_t b = q_desc + (uint64_t)((c0 * kQChunkBytes) >> 4);
+          mma_run_qk(d, a, b, id_qk, s == 0 ? 0u : 1u, two ? 1u : 0u);
+          umma_commit(&sh->kempty[slot]);
+          next_slot();
+        }
+        umma_commit(&sh->sfull[buf]);
+        ++sidx;
+        issued = true;
+        return true;
+      };
+      auto pv_mid = [&]() -> bool {
+        if (!mbar_wait_spin(&sh->pfull, npv & 1, lim)) return false;
+        tc_fence_after();
+        for (int c = 0; c < p.nvc; ++c) {
+          if (!mbar_wait_spin(&sh->vfull[slot], ph, lim)) return false;  // TMA stage
+          const uint64_t a0 = ring_desc_v + (uint64_t)((slot * kSlotBytes) >> 4);
+          pv_run(tmem + c * kH, a0, p_desc, id_pv, 1u);
+          umma_commit(&sh->vempty[slot]);
+          next_slot();
+        }
+        umma_commit(&sh->pvdone);
+        ++npv;
+        issued = true;
+        return true;
+      };
       auto pv = [&](bool first_tile) -> bool {
         if (!mbar_wait_spin(&sh->pfull, npv & 1, lim)) return false;
         tc_fence_after();
@@ -553,8 +591,10 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         const TokenPlan tp = plan_token<kSparse>(p, t, false);
         if (!tp.ok || tp.ntile == 0) continue;
         if (!is_pv) {
-          for (int i = 0; i < tp.ntile; ++i)
-            if (!qk(i == 0, i + 1 == tp.ntile)) { stop = true; break; }
+          for (int i = 0; i < tp.ntile; ++i) {
+            const bool ok2 = (i > 0 && i + 1 < tp.ntile) ? qk_mid() : qk(i == 0, i + 1 == tp.ntile);
+            if (!ok2) { stop = true; break; }
+          }
           ++qtok;
         } else {
           // O^T of the previous token must have been read out before PV(0)
@@ -565,7 +605,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           }
           tc_fence_after();
           for (int i = 0; i < tp.ntile; ++i)
-            if (!pv(i == 0)) { stop = true; break; }
+            if (!(i > 0 ? pv_mid() : pv(true))) { stop = true; break; }
           if (stop) break;
           if (!kEarly) umma_commit(&sh->ofull);
           ++ntok;
