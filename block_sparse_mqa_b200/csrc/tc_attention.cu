@@ -295,12 +295,26 @@ __device__ __forceinline__ void umma_ss_if(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
+// NP K chunks with a compile-time first accumulate flag (the narrow-Dk
+// instantiations; see mma_run_qk).
+template <int NP, bool FIRST>
+__device__ __forceinline__ void mma_run(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc) {
+#pragma unroll
+  for (int pn = 0; pn < NP; ++pn)
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      umma_ss(d, a0 + (uint64_t)((pn * kPanel) >> 4) + 2 * k,
+              b0 + (uint64_t)((pn * kQChunkBytes) >> 4) + 2 * k, idesc,
+              (FIRST && pn == 0 && k == 0) ? 0u : 1u);
+}
+
 // One K stage: two K chunks (4 MMAs each, M=128 keys, N=64 heads, K=16)
 // into S^T at d; A = K panels 16 KB apart, B = Q chunks 8 KB apart.  The
 // second chunk is issued only when `two`; the chunk count and the first
-// accumulate flag are runtime values, with no branch between the MMAs
-// (removing the per-stage branches to templated variants: sparse 0.771 ->
-// 0.753 ms, SWA 0.408 -> 0.398 ms).
+// accumulate flag are runtime values, with no branch between the MMAs.  The
+// wide-Dk instantiations (Dk > 256) use this form (sparse 0.771 -> 0.753 ms,
+// SWA 0.408 -> 0.398 ms at Dk 576); the narrow ones the templated variants
+// above (this form measured ~6 % slower at Dk 192 / Dv 128).
 __device__ __forceinline__ void mma_run_qk(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc,
                                            uint32_t acc0, uint32_t two) {
 #pragma unroll
@@ -322,7 +336,16 @@ __device__ __forceinline__ void pv_run(uint32_t d, uint64_t a0, uint64_t b0, uin
             kk == 0 ? acc0 : 1u);
 }
 
-template <int kMode>
+// pv_run with a compile-time first accumulate flag (narrow-Dk instantiations).
+template <bool FIRST>
+__device__ __forceinline__ void pv_run_t(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < kTile / 16; ++kk)
+    umma_ss(d, a0 + (uint64_t)(kk * 128), b0 + (uint64_t)(kk * 128), idesc,
+            (FIRST && kk == 0) ? 0u : 1u);
+}
+
+template <int kMode, bool kWide>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap,
@@ -498,6 +521,15 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       };
       // S^T(tile) = K_tile . Q^T into S buffer sidx & 1.  Each ring stage
       // (two 64-column chunks) is one run of MMAs with no branch inside.
+      auto qk_stage = [&](uint32_t d, uint64_t a, uint64_t b, int s, bool two) {
+        if constexpr (kWide) {
+          mma_run_qk(d, a, b, id_qk, s == 0 ? 0u : 1u, two ? 1u : 0u);
+        } else if (s == 0) {
+          if (two) mma_run<2, true>(d, a, b, id_qk); else mma_run<1, true>(d, a, b, id_qk);
+        } else {
+          if (two) mma_run<2, false>(d, a, b, id_qk); else mma_run<1, false>(d, a, b, id_qk);
+        }
+      };
       auto qk = [&](bool first_tile, bool last_tile) -> bool {
         const uint32_t buf = sidx & 1, use = sidx >> 1;
         if (!mbar_wait_spin(&sh->sempty[buf], (use & 1) ^ 1, lim)) return false;
@@ -513,7 +545,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           }
           const uint64_t a = ring_desc_k + (uint64_t)((slot * kSlotBytes) >> 4);
           const uint64_t b = q_desc + (uint64_t)((c0 * kQChunkBytes) >> 4);
-          mma_run_qk(d, a, b, id_qk, s == 0 ? 0u : 1u, two ? 1u : 0u);
+          qk_stage(d, a, b, s, two);
           if (last_tile) {  // the token's last QK has read these Q chunks
             umma_commit(&sh->qempty[c0]);
             if (two) umma_commit(&sh->qempty[c0 + 1]);
@@ -529,7 +561,10 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
       // O^T += V_tile^T . P^T (waits for P of this tile); 8 MMAs per stage
       // A token's middle tiles (neither its first nor its last) run the same
       // stages without the first / last tile's q waits and releases, so that
-      // no branch on them sits between two stages' runs of MMAs.
+      // no branch on them sits between two stages' runs of MMAs (the wide-Dk
+      // instantiations; the narrow ones run every tile through qk / pv,
+      // which measured faster there: the issuing thread's code shape moves
+      // the Dk 192 / Dv 128 window kernel by ~6 %).
       auto qk_mid = [&]() -> bool {
         const uint32_t buf = sidx & 1, use = sidx >> 1;
         if (!mbar_wait_spin(&sh->sempty[buf], (use & 1) ^ 1, lim)) return false;
@@ -541,7 +576,7 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           if (!mbar_wait_spin(&sh->kfull[slot], ph, lim)) return false;  // TMA stage
           const uint64_t a = ring_desc_k + (uint64_t)((slot * kSlotBytes) >> 4);
           const uint64_t b = q_desc + (uint64_t)((c0 * kQChunkBytes) >> 4);
-          mma_run_qk(d, a, b, id_qk, s == 0 ? 0u : 1u, two ? 1u : 0u);
+          qk_stage(d, a, b, s, two);
           umma_commit(&sh->kempty[slot]);
           next_slot();
         }
@@ -576,7 +611,12 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
           }
           const uint64_t a0 = ring_desc_v + (uint64_t)((slot * kSlotBytes) >> 4);
           const uint32_t d = tmem + c * kH;
-          pv_run(d, a0, p_desc, id_pv, first_tile ? 0u : 1u);
+          if constexpr (kWide) {
+            pv_run(d, a0, p_desc, id_pv, first_tile ? 0u : 1u);
+          } else {
+            if (first_tile) pv_run_t<true>(d, a0, p_desc, id_pv);
+            else pv_run_t<false>(d, a0, p_desc, id_pv);
+          }
           umma_commit(&sh->vempty[slot]);
           next_slot();
         }
@@ -591,9 +631,15 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
         const TokenPlan tp = plan_token<kSparse>(p, t, false);
         if (!tp.ok || tp.ntile == 0) continue;
         if (!is_pv) {
-          for (int i = 0; i < tp.ntile; ++i) {
-            const bool ok2 = (i > 0 && i + 1 < tp.ntile) ? qk_mid() : qk(i == 0, i + 1 == tp.ntile);
-            if (!ok2) { stop = true; break; }
+          if constexpr (kWide) {
+            for (int i = 0; i < tp.ntile; ++i) {
+              const bool ok2 =
+                  (i > 0 && i + 1 < tp.ntile) ? qk_mid() : qk(i == 0, i + 1 == tp.ntile);
+              if (!ok2) { stop = true; break; }
+            }
+          } else {
+            for (int i = 0; i < tp.ntile; ++i)
+              if (!qk(i == 0, i + 1 == tp.ntile)) { stop = true; break; }
           }
           ++qtok;
         } else {
@@ -604,8 +650,13 @@ tc_attention_kernel(const __grid_constant__ CUtensorMap kmap,
             break;
           }
           tc_fence_after();
-          for (int i = 0; i < tp.ntile; ++i)
-            if (!(i > 0 ? pv_mid() : pv(true))) { stop = true; break; }
+          if constexpr (kWide) {
+            for (int i = 0; i < tp.ntile; ++i)
+              if (!(i > 0 ? pv_mid() : pv(true))) { stop = true; break; }
+          } else {
+            for (int i = 0; i < tp.ntile; ++i)
+              if (!pv(i == 0)) { stop = true; break; }
+          }
           if (stop) break;
           if (!kEarly) umma_commit(&sh->ofull);
           ++ntok;
@@ -1049,10 +1100,16 @@ cudaError_t launch_mode(const AttnArgs& a, int mode, const FullArgs* fa, long lo
   ap.gate_own = a.gate_own;
   ap.gate_prev = a.gate_prev;
   const int grid = p.total_tokens < sm_count() ? p.total_tokens : sm_count();
-  auto kern = mode == kModeSparse   ? tc_attention_kernel<kModeSparse>
-              : mode == kModeFull   ? tc_attention_kernel<kModeFull>
-              : mode == kModeSwaLayer ? tc_attention_kernel<kModeSwaLayer>
-                                    : tc_attention_kernel<kModeSwa>;
+  // the issuers' form of a QK stage is chosen per instantiation (Dk > 256:
+  // runtime flags, else templated variants)
+  auto kern = ap.nck > 4 ? (mode == kModeSparse     ? tc_attention_kernel<kModeSparse, true>
+                            : mode == kModeFull     ? tc_attention_kernel<kModeFull, true>
+                            : mode == kModeSwaLayer ? tc_attention_kernel<kModeSwaLayer, true>
+                                                    : tc_attention_kernel<kModeSwa, true>)
+                         : (mode == kModeSparse     ? tc_attention_kernel<kModeSparse, false>
+                            : mode == kModeFull     ? tc_attention_kernel<kModeFull, false>
+                            : mode == kModeSwaLayer ? tc_attention_kernel<kModeSwaLayer, false>
+                                                    : tc_attention_kernel<kModeSwa, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
