@@ -141,27 +141,33 @@ __device__ __forceinline__ bool rendezvous(Shared* sh, int wg, uint32_t& ph, lon
   return ok;
 }
 
-// NP 64-column chunks of a K-major A stage (panels 16 KB apart) against B
-// chunks 8 KB apart: 4 MMAs (M = 128, N = 64, K = 16) per chunk into d.
-template <int NP, bool FIRST>
-__device__ __forceinline__ void kmajor_run(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc) {
+// One K-major stage: up to two 64-column chunks of the A stage (panels 16 KB
+// apart) against B chunks 8 KB apart, 4 MMAs (M = 128, N = 64, K = 16) per
+// chunk into d.  The first accumulate flag and whether the second chunk is
+// issued are runtime values (a guard predicate, not a branch between MMA
+// runs: 1.66 -> 1.62 ms block-sparse, 0.99 -> 0.96 ms window).
+__device__ __forceinline__ void kmajor_run_rt(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                              uint32_t acc0, uint32_t two) {
 #pragma unroll
-  for (int pn = 0; pn < NP; ++pn)
+  for (int k = 0; k < 4; ++k) umma_ss(d, a0 + 2 * k, b0 + 2 * k, idesc, k == 0 ? acc0 : 1u);
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      umma_ss(d, a0 + (uint64_t)((pn * kPanel) >> 4) + 2 * k,
-              b0 + (uint64_t)((pn * kChunkBytes) >> 4) + 2 * k, idesc,
-              (FIRST && pn == 0 && k == 0) ? 0u : 1u);
+  for (int k = 0; k < 4; ++k)
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %5, 0;\n\t"
+        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a0 + (uint64_t)(kPanel >> 4) + 2 * k), "l"(b0 + (uint64_t)(kChunkBytes >> 4) + 2 * k),
+        "r"(idesc), "r"(1u), "r"(two)
+        : "memory");
 }
-
 // One 128-row Dk chunk of dQ^T (+)= K_tile^T (MN-major, two 64-row panels)
-// . dS^T (MN-major) over 128 keys: 8 MMAs of 16 keys.
-template <bool FIRST>
-__device__ __forceinline__ void mnmajor_run(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc) {
+// . dS^T (MN-major) over 128 keys: 8 MMAs of 16 keys; acc0 = 0 opens it.
+__device__ __forceinline__ void mnmajor_run_rt(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                               uint32_t acc0) {
 #pragma unroll
   for (int kk = 0; kk < kTile / 16; ++kk)
-    umma_ss(d, a0 + (uint64_t)(kk * 128), b0 + (uint64_t)(kk * 128), idesc,
-            (FIRST && kk == 0) ? 0u : 1u);
+    umma_ss(d, a0 + (uint64_t)(kk * 128), b0 + (uint64_t)(kk * 128), idesc, kk == 0 ? acc0 : 1u);
 }
 
 template <bool kSparse>
@@ -371,11 +377,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
           }
           const uint64_t a = ring_k + (uint64_t)((slot * kSlotBytes) >> 4);
           const uint64_t b = bdesc + (uint64_t)((c0 * kChunkBytes) >> 4);
-          if (s == 0) {
-            if (two) kmajor_run<2, true>(d, a, b, id_k); else kmajor_run<1, true>(d, a, b, id_k);
-          } else {
-            if (two) kmajor_run<2, false>(d, a, b, id_k); else kmajor_run<1, false>(d, a, b, id_k);
-          }
+          kmajor_run_rt(d, a, b, id_k, s == 0 ? 0u : 1u, two ? 1u : 0u);
           if (last_tile) {
             umma_commit(&emptyc[c0]);
             if (two) umma_commit(&emptyc[c0 + 1]);
@@ -403,8 +405,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
           if (!mbar_wait_spin(&sh->full[slot], ph, lim)) return false;
           const uint64_t a0 = ring_mn + (uint64_t)((slot * kSlotBytes) >> 4);
           const uint32_t d = tmem + m * kH;
-          if (first_tile) mnmajor_run<true>(d, a0, ds_desc, id_mn);
-          else mnmajor_run<false>(d, a0, ds_desc, id_mn);
+          mnmajor_run_rt(d, a0, ds_desc, id_mn, first_tile ? 0u : 1u);
           umma_commit(&sh->empty[slot]);
           next_slot();
         }
