@@ -381,16 +381,32 @@ tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap kmap,
               if (!mbar_wait_spin(&sh->pds_full, m & 1, lim)) { ok = false; break; }
               tc_fence_after();
               const uint32_t first = any ? 1u : 0u;
-              for (int c = 0; c < nmc; ++c) {
+              auto acc_run = [&](int c) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                   umma_ss(tmem + col_acc + c * kKT,
                           a_mn + (uint64_t)((2 * c * kTokChunk) >> 4) + (uint64_t)(k * 128),
                           b_pd + (uint64_t)(k * 64), id_acc, (k == 0) ? first : 1u);
-                // this chunk pair of q_t (or dout_t) is read: the next member's
-                // copies may land there
-                umma_commit(&free_b[2 * c]);
-                if (2 * c + 1 < nch) umma_commit(&free_b[2 * c + 1]);
+              };
+              if (nch == 9 || nch == 8) {  // Dk 576 / 512, Dv 512: unrolled (-3 %)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                  acc_run(c);
+                  // this chunk pair of q_t (or dout_t) is read: the next
+                  // member's copies may land there
+                  umma_commit(&free_b[2 * c]);
+                  umma_commit(&free_b[2 * c + 1]);
+                }
+                if (nch == 9) {
+                  acc_run(4);
+                  umma_commit(&free_b[8]);
+                }
+              } else {
+                for (int c = 0; c < nmc; ++c) {
+                  acc_run(c);
+                  umma_commit(&free_b[2 * c]);
+                  if (2 * c + 1 < nch) umma_commit(&free_b[2 * c + 1]);
+                }
               }
               umma_commit(&sh->pds_free);
               any = true;
