@@ -281,7 +281,6 @@ __device__ __forceinline__ bool rendezvous(Shared* sh, int wg, uint32_t& ph, lon
   return ok;
 }
 
-
 // An SS MMA issued only when `on` (a guard predicate on the instruction,
 // not a branch around it).
 __device__ __forceinline__ void umma_ss_if(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -313,8 +312,9 @@ __device__ __forceinline__ void mma_run(uint32_t d, uint64_t a0, uint64_t b0, ui
 // second chunk is issued only when `two`; the chunk count and the first
 // accumulate flag are runtime values, with no branch between the MMAs.  The
 // wide-Dk instantiations (Dk > 256) use this form (sparse 0.771 -> 0.753 ms,
-// SWA 0.408 -> 0.398 ms at Dk 576); the narrow ones the templated variants
-// above (this form measured ~6 % slower at Dk 192 / Dv 128).
+// SWA 0.408 -> 0.398 ms at Dk 576); the narrow ones keep the earlier issuer
+// code with the templated variants above (the wide code measured ~6 %
+// slower at Dk 192 / Dv 128).
 __device__ __forceinline__ void mma_run_qk(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc,
                                            uint32_t acc0, uint32_t two) {
 #pragma unroll
