@@ -419,6 +419,38 @@ tc_block_score_kernel(const __grid_constant__ CUtensorMap kmap,
           }
           tc_fence_after();
           const uint32_t d = tmem + kSCol + r * 128;
+          if (p.nck == 9 && p.nq_smem > 0) {
+            // Dk 576: the key tile's three stages written out, no dispatch
+            // branch between their runs of MMAs
+            auto stage_wait = [&](int& slo) -> bool {
+              slo = r * kSlots + (int)kst;
+              return mbar_wait_spin(&sh->kfull[slo], kph, lim);
+            };
+            int sl;
+            if (!stage_wait(sl)) { ok = false; break; }
+            issue_stage<true, false>(d, tmem, 0, 0,
+                                     stage_desc0 + (uint64_t)((sl * kStageBytes) >> 4), idesc);
+            umma_commit(&sh->kempty[sl]);
+            next_slot();
+            if (!stage_wait(sl)) { ok = false; break; }
+            issue_stage<false, false>(d, tmem, 3, 0,
+                                      stage_desc0 + (uint64_t)((sl * kStageBytes) >> 4), idesc);
+            umma_commit(&sh->kempty[sl]);
+            next_slot();
+            if (!stage_wait(sl)) { ok = false; break; }
+            if (!qhi_seen) {
+              if (!mbar_wait(&sh->qhi_full, qtile & 1, lim)) { ok = false; break; }
+              qhi_seen = true;
+            }
+            issue_stage<false, true>(d, tmem, 6, qhi_desc[0],
+                                     stage_desc0 + (uint64_t)((sl * kStageBytes) >> 4), idesc);
+            umma_commit(&sh->kempty[sl]);
+            next_slot();
+            issued = true;
+            umma_commit(&sh->sfull[r]);
+            ++myidx;
+            continue;
+          }
           for (int st = 0; st < spt; ++st) {
             const int sl = r * kSlots + (int)kst;
             if (!mbar_wait_spin(&sh->kfull[sl], kph, lim)) {  // TMA stage (no fence needed)
